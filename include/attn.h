@@ -1,0 +1,151 @@
+/*
+ * attn.h -- C ABI of libattn_sm100.so: fused scaled-dot-product attention
+ * forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (exact attention; "FlashAttention-3" explainer, droidorbit.com,
+ * opening definition Softmax(Q K^T / sqrt(d)) V, with `scale` in place of
+ * 1/sqrt(d); causal masking as in "FlashAttention-3: como exprimir H100 al
+ * limite con atencion IO-aware", dibro.site, "Contribuciones clave"):
+ *
+ *   for every batch b, head h and query row i:
+ *     s_ij  = scale * <Q[b,h,i,:], K[b,h,j,:]>,  j in J_i
+ *     J_i   = {0 .. N-1}, or {0 .. i} when causal (queries and keys aligned)
+ *     O[b,h,i,:] = sum_j softmax_j(s_i.) V[b,h,j,:]
+ *     LSE[b,h,i] = ln sum_{j in J_i} exp(s_ij)
+ *
+ * computed tiled with online-softmax statistics (running max m, running sum
+ * l; dibro.site "Arquitectura y metodo"; droidorbit.com "Mathematical
+ * Formulation: The Online Softmax Rescaling Trick") so that the N x N score
+ * matrix is never written to device memory.
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ *  - Layout: every tensor is contiguous row-major [B][H][N][d] (head dim
+ *    innermost, the (batch, head, sequence, dim) stride order of the pages'
+ *    kernel signature); LSE is contiguous [B][H][N] fp32, natural log.
+ *  - Pointers are DEVICE pointers on the current CUDA device, 16-byte aligned
+ *    (TMA requirement).  The caller owns every buffer; the library never
+ *    frees or keeps them.  Outputs must not alias inputs.
+ *  - The library allocates no per-call device memory.  On first use of a
+ *    device it allocates one 16-byte status word (kept until exit).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous: they validate, enqueue and return.
+ *  - Validation happens before any launch; on failure nothing is enqueued and
+ *    the call returns ATTN_ERR_INVALID_ARG / ATTN_ERR_UNSUPPORTED /
+ *    ATTN_ERR_MISALIGNED.  Launch failures return ATTN_ERR_CUDA.  No C++
+ *    exception, abort or device trap crosses this boundary.
+ *  - Every internal wait of the kernels is bounded (default 1 s, environment
+ *    variable ATTN_WAIT_LIMIT_MS).  A wait that runs out makes the kernel
+ *    record ATTN_ERR_TIMEOUT in the device status word and return; read it
+ *    with attn_last_status().
+ *  - Results are deterministic: the same inputs give bit-identical outputs.
+ */
+#ifndef ATTN_SM100_H_
+#define ATTN_SM100_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* null pointer, size < 1, overflow, bad scale  */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head dim or dtype this build does not handle */
+  ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned             */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed          */
+  ATTN_ERR_TIMEOUT = 5       /* a kernel wait ran out (read after sync)       */
+} attn_status_t;
+
+typedef enum {
+  ATTN_BF16 = 0,
+  ATTN_FP16 = 1
+} attn_dtype_t;
+
+/*
+ * attn_fwd -- 16-bit attention forward.
+ *   q, k, v : [B][H][N][d] bf16 or fp16 (per `dtype`), read only.
+ *   o       : [B][H][N][d] same dtype, written.
+ *   lse     : [B][H][N] fp32, written; may be NULL (then not written).
+ *   B, H, N : >= 1, B*H*N < 2^31.   d : 64 or 128 (256: ATTN_ERR_UNSUPPORTED
+ *             in this build).
+ *   scale   : finite and > 0 (usually 1/sqrt(d)).
+ *   causal  : 0 or 1 (key j visible to query i iff j <= i).
+ * Rounding: scores, statistics and accumulation are fp32; P is rounded to
+ * the input dtype before the P.V product; O is rounded to the input dtype.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int N, int d, float scale, int causal, int dtype,
+                       void* stream);
+
+/*
+ * attn_quant_fp8 -- per-block e4m3 quantisation with optional incoherent
+ * processing (quantum-bit repost "H100 utilisation 75% ... FlashAttention-3",
+ * third technical upgrade: block-wise quantisation and incoherent processing;
+ * "FlashAttention-3 (HE)", systems-analysis.info, "Technical innovations"
+ * item 3: rotate Q and K by a random orthogonal, e.g. Hadamard, matrix
+ * before quantising; QK^T is unchanged).
+ *   x       : [B][H][N][d] bf16 input, read only.
+ *   x8      : [B][H][N][d] e4m3fn codes (uint8), written.
+ *   descale : [B][H][ceil(N/128)] fp32, written: one factor per block of 128
+ *             rows x d of one (b, h); x ~= value(code) * descale.
+ *   hadamard: 0 = plain; 1 = rotate each row by R = diag(signs) H_d / sqrt(d)
+ *             (Sylvester H_d) before quantising.  Use it for Q and K only.
+ *   signs   : d fp32 values of +-1 (device pointer), or NULL for all +1.
+ *             Ignored when hadamard = 0.  Q and K must use the same signs.
+ *   d       : 64 or 128.
+ * Per block: amax = max |y|; s = amax / 448 in fp32 (s = 1 if amax = 0);
+ * code = e4m3_rn_satfinite(y / s) with an IEEE fp32 division.
+ */
+attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int H, int N,
+                             int d, int hadamard, const float* signs, void* stream);
+
+/*
+ * attn_fwd_fp8 -- e4m3 attention forward (dibro.site "Arquitectura y metodo":
+ * FP8 attention with in-line per-block quantisation; quantum-bit repost,
+ * FP8 paragraph).
+ *   q8, k8, v8 : [B][H][N][d] e4m3fn codes from attn_quant_fp8 (Q and K
+ *                rotated with the same signs, or both unrotated; V never
+ *                rotated).
+ *   q_descale, k_descale, v_descale : [B][H][ceil(N/128)] fp32 factors.
+ *   o   : [B][H][N][d] bf16, written.   lse : [B][H][N] fp32 or NULL.
+ *   d   : 128 in this build (64 -> ATTN_ERR_UNSUPPORTED).
+ *   v_transpose : 0 = feed V to the tensor core MN-major, straight from the
+ *                 TMA tile; 1 = transpose each V tile in shared memory to
+ *                 K-major first (the pages' layout step; sm_100a accepts
+ *                 either, both give identical results).
+ * Scores use scale * q_descale * k_descale per (query block, key block);
+ * P is rounded to e4m3 after multiplying by 256 * v_descale[j] / max_j
+ * v_descale[j]; statistics are fp32 and l sums the unrounded P.
+ */
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                           const float* q_descale, const float* k_descale,
+                           const float* v_descale, void* o, float* lse, int B, int H, int N,
+                           int d, float scale, int causal, int v_transpose, void* stream);
+
+/*
+ * attn_last_status -- synchronises `stream`, then reads and clears the
+ * current device's status word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT (a kernel
+ * wait ran out; the affected outputs are undefined) or ATTN_ERR_CUDA.
+ * `where` (may be NULL) receives 2 ints: the barrier id and block index
+ * recorded with the error.
+ */
+attn_status_t attn_last_status(void* stream, int* where);
+
+/* Static description of a status code. */
+const char* attn_status_string(attn_status_t s);
+
+/*
+ * attn_debug_set_fault -- test hook for the bounded waits.  When `mode` is 1
+ * the next attn_fwd launch runs with its TMA producer told to skip its first
+ * load-complete arrival, so the consumers' waits must run out: the call
+ * returns ATTN_OK and attn_last_status() then reports ATTN_ERR_TIMEOUT.  The
+ * hook resets itself after one launch.  `wait_limit_ms` (> 0) overrides the
+ * wait limit for that launch.  No device fault, trap or hang is involved.
+ */
+attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_SM100_H_ */

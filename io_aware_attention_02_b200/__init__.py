@@ -9,12 +9,14 @@ The binding is imported lazily so that ``inputs`` (the seeded generator) can
 be used on machines without the built library.
 """
 
-__all__ = ["fwd", "fwd_fp8", "quant_fp8", "lib"]
+import importlib
+
+__all__ = ["fwd", "fwd_fp8", "quant_fp8", "binding", "inputs"]
 
 
 def __getattr__(name):
-    if name in ("fwd", "fwd_fp8", "quant_fp8", "lib", "binding"):
-        from . import binding
-
-        return binding if name == "binding" else getattr(binding, name)
+    if name in ("binding", "inputs", "build"):
+        return importlib.import_module(f"{__name__}.{name}")
+    if name in ("fwd", "fwd_fp8", "quant_fp8"):
+        return getattr(importlib.import_module(f"{__name__}.binding"), name)
     raise AttributeError(name)

@@ -1,0 +1,168 @@
+"""ctypes binding of libattn_sm100.so (C ABI in include/attn.h).
+
+Argument marshalling only: torch provides device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no fallback: if the library cannot be loaded, or a GPU is missing,
+these functions raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libattn_sm100.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(6)
+ATTN_BF16, ATTN_FP16 = 0, 1
+
+# name -> (restype, argtypes); mirrors include/attn.h
+_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_quant_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_last_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
+    "attn_status_string": (ctypes.c_char_p, [_I]),
+    "attn_debug_set_fault": (_I, [_I, _I]),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {code} ({status_string(code)})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once) and set every exported signature."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m io_aware_attention_02_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def lib() -> ctypes.CDLL:
+    return load()
+
+
+def status_string(code: int) -> str:
+    return load().attn_status_string(int(code)).decode()
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn: str, code: int):
+    if code != ATTN_OK:
+        raise AttnError(fn, code)
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D [B, H, N, d]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: float | None = None, out: torch.Tensor | None = None,
+        lse: torch.Tensor | None = None, return_lse: bool = True):
+    """O, LSE = attention(q, k, v) through ``attn_fwd`` on the current stream.
+
+    q, k, v: contiguous CUDA tensors [B, H, N, d] of bf16 or fp16.
+    Returns (o, lse) with lse fp32 [B, H, N] (None if ``return_lse`` is False).
+    """
+    _check_qkv(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bf16 or all fp16")
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
+    code = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse) if return_lse else None,
+                           B, H, N, d, scale, int(bool(causal)), dtype, _stream(q.device))
+    _check("attn_fwd", code)
+    return o, (lse if return_lse else None)
+
+
+def quant_fp8(x: torch.Tensor, hadamard: bool = False, signs: torch.Tensor | None = None,
+              out: torch.Tensor | None = None, descale: torch.Tensor | None = None):
+    """Per-block e4m3 quantisation through ``attn_quant_fp8``.
+
+    Returns (codes uint8 [B, H, N, d], descale fp32 [B, H, ceil(N/128)]).
+    """
+    if not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("x must be a contiguous CUDA bf16 tensor [B, H, N, d]")
+    B, H, N, d = x.shape
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    if descale is None:
+        descale = torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    if signs is not None:
+        signs = signs.to(device=x.device, dtype=torch.float32).contiguous()
+    code = load().attn_quant_fp8(_ptr(x), _ptr(codes), _ptr(descale), B, H, N, d,
+                                 int(bool(hadamard)), _ptr(signs) if hadamard else None,
+                                 _stream(x.device))
+    _check("attn_quant_fp8", code)
+    return codes, descale
+
+
+def fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal: bool = False,
+            scale: float | None = None, v_transpose: bool = False, out=None, lse=None,
+            return_lse: bool = True):
+    """O (bf16), LSE = e4m3 attention through ``attn_fwd_fp8``.
+
+    q8, k8, v8: uint8 e4m3 codes [B, H, N, d] from :func:`quant_fp8`;
+    descales fp32 [B, H, ceil(N/128)].
+    """
+    _check_qkv(q8, k8, v8)
+    B, H, N, d = q8.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    code = load().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_descale), _ptr(k_descale),
+                               _ptr(v_descale), _ptr(o), _ptr(lse) if return_lse else None,
+                               B, H, N, d, scale, int(bool(causal)), int(bool(v_transpose)),
+                               _stream(q8.device))
+    _check("attn_fwd_fp8", code)
+    return o, (lse if return_lse else None)
+
+
+def last_status(stream=None):
+    """(status code, [barrier id, block index]) of the current device; clears it."""
+    where = (ctypes.c_int * 2)()
+    s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    code = load().attn_last_status(ctypes.c_void_p(s), where)
+    return code, [where[0], where[1]]
+
+
+def debug_set_fault(mode: int, wait_limit_ms: int = 0):
+    _check("attn_debug_set_fault", load().attn_debug_set_fault(int(mode), int(wait_limit_ms)))

@@ -1,0 +1,274 @@
+// C ABI of libattn_sm100.so (declared in include/attn.h): argument
+// validation, TMA descriptor construction, kernel selection and launch.
+// Host code only marshals; every step of the attention runs in the kernels.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "fwd_sm100.cuh"
+#include "quant_fp8.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  int* status = nullptr;  // 4 ints, see ptx.cuh
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+int g_fault_mode = 0;
+int g_fault_limit_ms = 0;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device lazily created state: status word and SM count.
+attn_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (st.status == nullptr) {
+    if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    int* p = nullptr;
+    if (cudaMalloc(&p, 4 * sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemset(p, 0, 4 * sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    st.status = p;
+  }
+  *out = &st;
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D tiled map over a contiguous [BH][N][D] tensor: box = (box_cols, 128, 1),
+// 128-byte swizzle; out-of-range rows read as zero.
+attn_status_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize,
+                       int BH, int N, int D, int box_cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esize,
+                           static_cast<cuuint64_t>(N) * D * esize};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+unsigned long long wait_limit_ns() {
+  static unsigned long long ns = [] {
+    const char* e = std::getenv("ATTN_WAIT_LIMIT_MS");
+    long ms = e ? std::strtol(e, nullptr, 10) : 0;
+    if (ms <= 0) ms = 1000;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+attn_status_t common_checks(int B, int H, int N, float scale, int causal) {
+  if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <typename E, int D, bool CAUSAL>
+attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
+  using Cfg = attn::FwdCfg<E, D>;
+  auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL>;
+  static bool attr_done = false;  // per instance; set once per process
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_done = true;
+  }
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename E, int D>
+attn_status_t launch_fwd_c(const attn::FwdParams& p, int grid, int causal, cudaStream_t s) {
+  return causal ? launch_fwd<E, D, true>(p, grid, s) : launch_fwd<E, D, false>(p, grid, s);
+}
+
+// Fills the fields shared by the 16-bit and FP8 launches.
+attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void* o, int BH, int N,
+                          float scale) {
+  p->o = o;
+  p->lse = lse;
+  p->status = st->status;
+  p->BH = BH;
+  p->N = N;
+  p->n_kv = (N + 127) / 128;
+  p->n_qpairs = (N + 255) / 256;
+  p->n_units = BH * p->n_qpairs;
+  p->scale_log2 = scale * 1.4426950408889634f;
+  p->wait_limit_ns = wait_limit_ns();
+  std::lock_guard<std::mutex> lock(g_mu);
+  p->fault = g_fault_mode;
+  if (g_fault_mode != 0 && g_fault_limit_ms > 0)
+    p->wait_limit_ns = static_cast<unsigned long long>(g_fault_limit_ms) * 1000000ull;
+  g_fault_mode = 0;
+  g_fault_limit_ms = 0;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported head dim or dtype";
+    case ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms) {
+  if (mode < 0 || mode > 1 || wait_limit_ms < 0) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_fault_mode = mode;
+  g_fault_limit_ms = wait_limit_ms;
+  return ATTN_OK;
+}
+
+attn_status_t attn_last_status(void* stream, int* where) {
+  DeviceState* st = nullptr;
+  attn_status_t r = device_state(&st);
+  if (r != ATTN_OK) return r;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(h, st->status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemset(st->status, 0, sizeof(h)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (where != nullptr) {
+    where[0] = h[1];
+    where[1] = h[2];
+  }
+  if (h[0] == 0) return ATTN_OK;
+  return h[0] == ATTN_ERR_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, float scale, int causal, int dtype, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+
+  DeviceState* st = nullptr;
+  if ((r = device_state(&st)) != ATTN_OK) return r;
+
+  const int BH = B * H;
+  const CUtensorMapDataType dt =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  attn::FwdParams p{};
+  if ((r = make_map(&p.tm_q, q, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  fill_common(&p, st, lse, o, BH, N, scale);
+  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == ATTN_BF16)
+    return d == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
+                   : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
+  return d == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
+                 : launch_fwd_c<__half, 128>(p, grid, causal, s);
+}
+
+attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int H, int N, int d,
+                             int hadamard, const float* signs, void* stream) {
+  if (x == nullptr || x8 == nullptr || descale == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || static_cast<long long>(B) * H * N >= (1ll << 31))
+    return ATTN_ERR_INVALID_ARG;
+  if (hadamard != 0 && hadamard != 1) return ATTN_ERR_INVALID_ARG;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(descale) & 3u) != 0 ||
+      (signs != nullptr && (reinterpret_cast<uintptr_t>(signs) & 3u) != 0))
+    return ATTN_ERR_MISALIGNED;
+  const int nb = (N + 127) / 128;
+  const int grid = nb * B * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* q8 = static_cast<uint8_t*>(x8);
+  if (d == 64)
+    attn::attn_quant_fp8_kernel<64><<<grid, 256, 0, s>>>(xb, q8, descale, signs, N, nb, hadamard);
+  else
+    attn::attn_quant_fp8_kernel<128><<<grid, 256, 0, s>>>(xb, q8, descale, signs, N, nb, hadamard);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_descale,
+                           const float* k_descale, const float* v_descale, void* o, float* lse,
+                           int B, int H, int N, int d, float scale, int causal, int v_transpose,
+                           void* stream) {
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || o == nullptr || q_descale == nullptr ||
+      k_descale == nullptr || v_descale == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (v_transpose != 0 && v_transpose != 1) return ATTN_ERR_INVALID_ARG;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (v_transpose != 0) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(q_descale) | reinterpret_cast<uintptr_t>(k_descale) |
+                       reinterpret_cast<uintptr_t>(v_descale) |
+                       (lse ? reinterpret_cast<uintptr_t>(lse) : 0);
+  if ((a4 & 3u) != 0) return ATTN_ERR_MISALIGNED;
+
+  DeviceState* st = nullptr;
+  if ((r = device_state(&st)) != ATTN_OK) return r;
+  const int BH = B * H;
+  attn::FwdParams p{};
+  const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if ((r = make_map(&p.tm_q, q8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
+  p.q_desc = q_descale;
+  p.k_desc = k_descale;
+  p.v_desc = v_descale;
+  fill_common(&p, st, lse, o, BH, N, scale);
+  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  return launch_fwd_c<__nv_fp8_e4m3, 128>(p, grid, causal, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

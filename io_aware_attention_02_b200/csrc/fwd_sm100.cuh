@@ -1,0 +1,498 @@
+// Fused attention forward for sm_100a, 16-bit inputs (bf16 / fp16), head dim
+// 64 or 128, optional causal mask.
+//
+// What it computes (exact attention, the definition Softmax(Q K^T / sqrt(d)) V
+// of the "FlashAttention-3" explainer on droidorbit.com, with `scale` in place
+// of 1/sqrt(d)), tiled as in "FlashAttention-3: como exprimir H100 al limite
+// con atencion IO-aware" (dibro.site), "Arquitectura y metodo": Q in 128-row
+// tiles, K/V in 128-row tiles, the running max m and sum l kept per row, the
+// output rescaled by exp2(m_old - m_new) ("Mathematical Formulation: The
+// Online Softmax Rescaling Trick", droidorbit.com) and divided by l once at
+// the end.  The N x N score matrix never leaves the SM: S lives in tensor
+// memory, P overwrites it in place as 16-bit values.
+//
+// Structure (Blackwell-native; the pages' Hopper WGMMA design is prior art):
+//   * persistent grid, one CTA per SM, work unit = (batch*head, 256 query rows)
+//     = two 128-row Q tiles ("slots");
+//   * warp 0: TMA producer -- Q tiles once per unit, then K_j, V_j through a
+//     multi-stage shared-memory ring guarded by full/empty mbarriers
+//     (producer/consumer warp specialisation: dibro.site, "Arquitectura y
+//     metodo" item 3; quantum-bit repost, first technical upgrade);
+//   * warp 1: one thread issues every tcgen05.mma -- S_t = Q_t K_j^T
+//     (SMEM x SMEM -> TMEM) and O_t += P_t V_j (P from TMEM, V from SMEM);
+//   * warps 2-5 / 6-9: softmax warpgroups, one per Q tile, one thread per
+//     query row.  While one group turns S into P the tensor core works on the
+//     other tile: the ping-pong schedule of the quantum-bit repost
+//     ("ping-pong scheduling") carried over to tcgen05;
+//   * causal: key tiles entirely above the diagonal are never loaded or
+//     multiplied (dibro.site, "Contribuciones clave"); the diagonal tile and a
+//     ragged last tile are masked element-wise;
+//   * the running max is only raised when it grows by more than 2^8 (lazy
+//     rescaling); the final division by l keeps the result exact up to
+//     rounding while O is rescaled only on the rare large jumps.
+//
+// The same pipeline runs the FP8 (e4m3) variant (dibro.site, "Arquitectura
+// y metodo": FP8 with in-line per-block quantisation; quantum-bit repost, FP8
+// paragraph): tcgen05 kind::f8f6f4 products, scores scaled per (query block,
+// key block) by the blocks' descale factors, P rounded to e4m3 after a
+// power-of-two gain (256) times v_descale[j] / max v_descale, statistics and
+// accumulators in fp32 (vikram-blog.pages.dev, "Production Gotchas": softmax
+// accumulators stay fp32 under FP8), O divided by 256 * l / max v_descale at
+// the end.
+//
+// Every mbarrier wait is bounded (timeout -> status word, no trap, no hang).
+#pragma once
+#include <cuda_fp8.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+// Element traits: bytes per value, tcgen05 kind, operand format code.
+template <typename E>
+struct Elem;
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  static constexpr bool kF8 = false;
+  static constexpr uint32_t kFmt = 1;   // kind::f16 BF16
+  using Out = __nv_bfloat16;
+};
+template <>
+struct Elem<__half> {
+  static constexpr int kBytes = 2;
+  static constexpr bool kF8 = false;
+  static constexpr uint32_t kFmt = 0;   // kind::f16 F16
+  using Out = __half;
+};
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr int kBytes = 1;
+  static constexpr bool kF8 = true;
+  static constexpr uint32_t kFmt = 0;   // kind::f8f6f4 E4M3
+  using Out = __nv_bfloat16;
+};
+
+struct FwdParams {
+  CUtensorMap tm_q;  // 3-D maps over [BH][N][D], 64-column (128-byte) boxes, 128-byte swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  void* o;           // [BH][N][D] 16-bit output
+  float* lse;        // [BH][N] natural-log LSE, may be null
+  const float* q_desc;  // FP8 only: [BH][n_kv] descale factors per 128-row block
+  const float* k_desc;
+  const float* v_desc;
+  int* status;       // 4-int device status word
+  int BH, N, n_kv, n_qpairs, n_units;
+  float scale_log2;  // scale * log2(e)
+  unsigned long long wait_limit_ns;
+  int fault;         // test hook: 1 = CTA 0 skips its first K load (waits must run out)
+};
+
+template <typename E, int D>
+struct FwdCfg {
+  static constexpr int kTileRows = 128;
+  static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int kChunkCols = 128 / Elem<E>::kBytes;
+  static constexpr int kChunks = D * Elem<E>::kBytes / 128;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (kTileBytes <= 16384) ? 8 : 4;
+  static constexpr int kKeysPerMma = 32 / Elem<E>::kBytes;  // 32 bytes of K per tcgen05.mma
+  static constexpr int kThreads = 320;
+  static constexpr int kTmemCols = 512;                   // S0 | S1 | O0 | O1
+  static constexpr int kColS = 0;                         // + t * 128
+  static constexpr int kColO = 256;                       // + t * D
+  // dynamic shared memory: [Q0 | Q1 | ring of kStages tiles | barriers]
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + 1 KiB alignment slack
+};
+
+// Barrier ids reported on timeout (status[1]).
+enum : int {
+  kWhereQEmpty = 1, kWhereKvEmpty = 2, kWhereQFull = 3, kWhereKvFull = 4,
+  kWherePFull = 5, kWhereSFull = 6, kWhereOFull = 7, kWhereDrain = 8
+};
+
+template <typename E, int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
+  using Cfg = FwdCfg<E, D>;
+  using T = typename Elem<E>::Out;
+  constexpr bool kF8 = Elem<E>::kF8;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + Cfg::kOffQ;
+  uint8_t* sKV = smem + Cfg::kOffKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* s_full = bars + 2;       // [2]
+  uint64_t* p_full = bars + 4;       // [2]
+  uint64_t* o_full = bars + 6;       // [2]
+  uint64_t* drain = bars + 8;
+  uint64_t* kv_full = bars + 9;      // [S]
+  uint64_t* kv_empty = bars + 9 + S; // [S]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * S);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, 128);
+      mbar_init(o_full + t, 1);
+    }
+    mbar_init(drain, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_kv = p.n_kv;
+  const unsigned long long lim = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      uint32_t kv_iter = 0, unit_iter = 0;
+      int64_t skipped = -1;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
+        const int bh = unit / p.n_qpairs;
+        const int qr = unit % p.n_qpairs;
+        const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+        const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
+        ok = mbar_wait(q_empty, (unit_iter & 1) ^ 1, p.status, abort_flag, kWhereQEmpty, lim);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, 2 * Cfg::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_3d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_q, q_full,
+                        c * Cfg::kChunkCols, qp * 256 + t * 128, bh);
+        for (int j = 0; j < n1 && ok; ++j) {
+          for (int which = 0; which < 2; ++which, ++kv_iter) {
+            const uint32_t s = kv_iter % S;
+            ok = mbar_wait(kv_empty + s, ((kv_iter / S) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
+            if (!ok) break;
+            if (p.fault == 1 && blockIdx.x == 0 && kv_iter == 0) {
+              skipped = 0;  // test hook: this stage never completes
+              continue;
+            }
+            mbar_arrive_expect_tx(kv_full + s, Cfg::kTileBytes);
+            const CUtensorMap* map = which == 0 ? &p.tm_k : &p.tm_v;
+            for (int c = 0; c < Cfg::kChunks; ++c)
+              tma_load_3d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
+                          c * Cfg::kChunkCols, j * 128, bh);
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA may exit: wait
+        // for each ring stage's last armed phase and for the last Q load.
+        volatile int never = 0;
+        for (uint32_t i = (kv_iter > S ? kv_iter - S : 0); i < kv_iter; ++i)
+          if (static_cast<int64_t>(i) != skipped) mbar_wait(kv_full + (i % S), (i / S) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+        if (unit_iter > 0) mbar_wait(q_full, (unit_iter - 1) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t fmt = Elem<E>::kFmt;
+      constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, 0, 128, 128);
+      constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 0, 1, 128, D);
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sKV_addr = smem_u32(sKV);
+      uint32_t kv_iter = 0, unit_iter = 0;
+      uint32_t p_cnt[2] = {0, 0};
+      bool ok = true;
+
+      auto issue_s = [&](int t, uint32_t kstage) {
+        const uint32_t a0 = sQ_addr + t * Cfg::kTileBytes;
+        const uint32_t b0 = sKV_addr + kstage * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
+          // K-major, 128-byte swizzle: each product consumes 32 bytes of the
+          // head dim; four of them span one 128-byte chunk row.
+          const uint32_t off = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
+          mma_ss(tmem + Cfg::kColS + t * 128, smem_desc_sw128(a0 + off, 16, 1024),
+                 smem_desc_sw128(b0 + off, 16, 1024), idesc_s, kk > 0, kF8);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t vstage, bool acc) {
+        const uint32_t b0 = sKV_addr + vstage * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 128 / Cfg::kKeysPerMma; ++kk) {
+          // P_t: 128 rows x 128 keys packed in TMEM (32 bytes = 8 columns per
+          // product).  V_j: MN-major (head dim contiguous), kKeysPerMma keys
+          // = kKeysPerMma rows of 128 bytes per product.
+          mma_ts(tmem + Cfg::kColO + t * D, tmem + Cfg::kColS + t * 128 + kk * 8,
+                 smem_desc_sw128(b0 + kk * Cfg::kKeysPerMma * 128, Cfg::kChunkBytes, 1024), idesc_o,
+                 (acc || kk > 0) ? 1u : 0u, kF8);
+        }
+      };
+      auto wait_p = [&](int t) -> bool {
+        bool r = mbar_wait(p_full + t, p_cnt[t] & 1, p.status, abort_flag, kWherePFull, lim);
+        ++p_cnt[t];
+        tc_fence_after();
+        return r;
+      };
+      auto wait_kv = [&](uint32_t idx) -> bool {
+        bool r = mbar_wait(kv_full + (idx % S), (idx / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
+        tc_fence_after();
+        return r;
+      };
+
+      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
+        const int qr = unit % p.n_qpairs;
+        const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+        const int n0 = CAUSAL ? min(2 * qp + 1, n_kv) : n_kv;
+        const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
+        const uint32_t base = kv_iter;  // K_j at base + 2j, V_j at base + 2j + 1
+
+        ok = mbar_wait(q_full, unit_iter & 1, p.status, abort_flag, kWhereQFull, lim);
+        tc_fence_after();
+        if (!ok) break;
+        ok = wait_kv(base);
+        if (!ok) break;
+        issue_s(0, base % S);
+        mma_commit(s_full + 0);
+        issue_s(1, base % S);
+        mma_commit(s_full + 1);
+        mma_commit(kv_empty + (base % S));
+
+        for (int j = 1; j < n1 && ok; ++j) {
+          const uint32_t ik = base + 2 * j, iv = base + 2 * (j - 1) + 1;
+          if (!(ok = wait_kv(ik))) break;
+          if (!(ok = wait_kv(iv))) break;
+          if (j < n0) {
+            if (!(ok = wait_p(0))) break;
+            issue_pv(0, iv % S, j - 1 > 0);
+            issue_s(0, ik % S);
+            mma_commit(s_full + 0);
+          } else if (j == n0) {
+            if (!(ok = wait_p(0))) break;
+            issue_pv(0, iv % S, j - 1 > 0);
+            mma_commit(o_full + 0);
+          }
+          if (!(ok = wait_p(1))) break;
+          issue_pv(1, iv % S, j - 1 > 0);
+          mma_commit(kv_empty + (iv % S));
+          issue_s(1, ik % S);
+          mma_commit(s_full + 1);
+          mma_commit(kv_empty + (ik % S));
+        }
+        if (!ok) break;
+        const uint32_t iv = base + 2 * (n1 - 1) + 1;
+        if (!(ok = wait_kv(iv))) break;
+        if (n0 == n1) {
+          if (!(ok = wait_p(0))) break;
+          issue_pv(0, iv % S, n1 - 1 > 0);
+          mma_commit(o_full + 0);
+        }
+        if (!(ok = wait_p(1))) break;
+        issue_pv(1, iv % S, n1 - 1 > 0);
+        mma_commit(o_full + 1);
+        mma_commit(kv_empty + (iv % S));
+        mma_commit(q_empty);
+        kv_iter += 2 * n1;
+      }
+      if (!ok) {
+        // Wait for the MMAs already issued before TMEM is released.
+        mma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, nullptr, &never, kWhereDrain, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int t = (warp - 2) >> 2;                 // Q tile (slot) 0 or 1
+    const int quarter = warp & 3;                  // TMEM lane quarter this warp may access
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + Cfg::kColS + t * 128;
+    const uint32_t tO = tmem + lane_off + Cfg::kColO + t * D;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    // FP8: P is multiplied by this power of two before rounding to e4m3, and
+    // the max may lag the true max by at most kLazy (log2 units) so that
+    // P * gain <= 256 * 2^0.75 < 448 stays finite in e4m3.
+    constexpr float kPGain = 256.0f;
+    constexpr float kLazy = kF8 ? 0.75f : 8.0f;
+
+    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
+      const int bh = unit / p.n_qpairs;
+      const int qr = unit % p.n_qpairs;
+      const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+      const int nt = CAUSAL ? min(2 * qp + t + 1, n_kv) : n_kv;
+      const int row = qp * 256 + t * 128 + row_in_tile;
+      float m = -INFINITY, l = 0.f;
+      float cq = p.scale_log2;   // score -> log2 domain factor (times q descale for FP8)
+      float vmax = 1.0f;         // FP8: max v descale of this head
+      if constexpr (kF8) {
+        const size_t dbase = static_cast<size_t>(bh) * n_kv;
+        const int qblk = qp * 2 + t;
+        cq *= p.q_desc[dbase + min(qblk, n_kv - 1)];
+        float vm = 0.f;
+        for (int b = lane; b < n_kv; b += 32) vm = fmaxf(vm, p.v_desc[dbase + b]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+        vmax = vm;
+      }
+
+      for (int j = 0; j < nt; ++j) {
+        bool w = mbar_wait(s_full + t, s_cnt & 1, p.status, abort_flag, kWhereSFull, lim);
+        ++s_cnt;
+        if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+        tc_fence_after();
+
+        float c = cq;
+        float pgain = 1.0f;
+        if constexpr (kF8) {
+          const size_t dbase = static_cast<size_t>(bh) * n_kv;
+          c = cq * p.k_desc[dbase + j];
+          pgain = kPGain * __fdiv_rn(p.v_desc[dbase + j], vmax);
+        }
+
+        float s[128];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tS + cc * 32, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
+        }
+        tmem_wait_ld();
+
+        const int key0 = j * 128;
+        const bool need_mask = (CAUSAL && key0 + 127 > qp * 256 + t * 128) || (key0 + 128 > p.N);
+        if (need_mask) {
+          const int lim_key = CAUSAL ? min(row, p.N - 1) : (p.N - 1);
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (key0 + i > lim_key) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        mx *= c;
+        // Lazy max: raise m only when the tile max exceeds it by more than
+        // kLazy (log2 units); then alpha = 2^(m_old - m_new), 0 on the first
+        // tile.  The final division by l makes the stale max exact.
+        float alpha = 1.0f;
+        if (mx > m + kLazy) {
+          alpha = ex2_approx(m - mx);
+          m = mx;
+        }
+        const float neg_m = -m;
+        float sum = 0.f;
+        if constexpr (!kF8) {
+          // two halves of 64 keys -> 32 packed columns each, so that only
+          // half of P is live in registers at a time
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = ex2_approx(fmaf(s[64 * hf + 2 * i], c, neg_m));
+              const float p1 = ex2_approx(fmaf(s[64 * hf + 2 * i + 1], c, neg_m));
+              sum += p0 + p1;
+              pk[i] = pack2<T>(p0, p1);
+            }
+            tmem_st32(tS + 32 * hf, pk);
+          }
+        } else {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2_approx(fmaf(s[4 * i], c, neg_m));
+            const float p1 = ex2_approx(fmaf(s[4 * i + 1], c, neg_m));
+            const float p2 = ex2_approx(fmaf(s[4 * i + 2], c, neg_m));
+            const float p3 = ex2_approx(fmaf(s[4 * i + 3], c, neg_m));
+            sum += (p0 + p1) + (p2 + p3);
+            pk[i] = pack4_e4m3(p0 * pgain, p1 * pgain, p2 * pgain, p3 * pgain);
+          }
+          tmem_st32(tS, pk);
+        }
+        l = l * alpha + sum;
+        // Rescale O_t when some row of this warp raised its max.  The PV
+        // product of the previous key tile has completed: S_t(j) was
+        // committed after it.
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(tO + cc * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + cc * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + t);
+      }
+      if (!ok) break;
+
+      // ------------------------------------------------------------ epilogue
+      bool w = mbar_wait(o_full + t, o_cnt & 1, p.status, abort_flag, kWhereOFull, lim);
+      ++o_cnt;
+      if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+      tc_fence_after();
+      const float inv_l = kF8 ? __fdiv_rn(vmax, kPGain * l) : 1.0f / l;
+      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.N + row) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tO + cc * 32, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<T>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+        if (row < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (p.lse != nullptr && row < p.N)
+        p.lse[static_cast<size_t>(bh) * p.N + row] = (m + __log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+}  // namespace attn

@@ -1,0 +1,106 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/attn.h declares, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from io_aware_attention_02_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.LIB_PATH):
+        from io_aware_attention_02_b200 import build
+        build.build()
+    return binding.load()
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == sorted(["attn_fwd", "attn_quant_fp8", "attn_fwd_fp8", "attn_last_status",
+                                  "attn_status_string", "attn_debug_set_fault"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(binding.SIGNATURES) == set(_declared())
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert binding.status_string(code)
+    assert binding.status_string(99) == "unknown status"
+
+
+GOOD = 0x10000  # 16-byte-aligned fake address: never dereferenced, validation fails first
+
+
+def _fwd(lib, q=GOOD, k=GOOD, v=GOOD, o=GOOD, lse=None, B=1, H=1, N=128, d=64, scale=0.125,
+         causal=0, dtype=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), binding.ATTN_ERR_INVALID_ARG),
+    (dict(o=None), binding.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), binding.ATTN_ERR_INVALID_ARG),
+    (dict(N=0), binding.ATTN_ERR_INVALID_ARG),
+    (dict(H=-1), binding.ATTN_ERR_INVALID_ARG),
+    (dict(B=1 << 16, H=1 << 16, N=1), binding.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.ATTN_ERR_INVALID_ARG),
+    (dict(scale=-1.0), binding.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), binding.ATTN_ERR_INVALID_ARG),
+    (dict(d=0), binding.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), binding.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), binding.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=7), binding.ATTN_ERR_UNSUPPORTED),
+    (dict(q=GOOD + 8), binding.ATTN_ERR_MISALIGNED),
+    (dict(v=GOOD + 2), binding.ATTN_ERR_MISALIGNED),
+    (dict(lse=GOOD + 2), binding.ATTN_ERR_MISALIGNED),
+])
+def test_fwd_validation_before_any_cuda_call(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def test_quant_and_fp8_validation(lib):
+    Q = lib.attn_quant_fp8
+    assert Q(None, GOOD, GOOD, 1, 1, 128, 128, 0, None, None) == binding.ATTN_ERR_INVALID_ARG
+    assert Q(GOOD, GOOD, GOOD, 1, 1, 128, 128, 2, None, None) == binding.ATTN_ERR_INVALID_ARG
+    assert Q(GOOD, GOOD, GOOD, 1, 1, 128, 96, 0, None, None) == binding.ATTN_ERR_UNSUPPORTED
+    assert Q(GOOD + 4, GOOD, GOOD, 1, 1, 128, 128, 0, None, None) == binding.ATTN_ERR_MISALIGNED
+    F = lib.attn_fwd_fp8
+    args = [GOOD] * 8 + [1, 1, 128, 128, 0.1, 0, 0, None]
+    bad = list(args); bad[3] = None
+    assert F(*bad) == binding.ATTN_ERR_INVALID_ARG
+    bad = list(args); bad[11] = 64
+    assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
+    bad = list(args); bad[0] = GOOD + 1
+    assert F(*bad) == binding.ATTN_ERR_MISALIGNED
+    bad = list(args); bad[14] = 3
+    assert F(*bad) == binding.ATTN_ERR_INVALID_ARG
+
+
+def test_debug_hook_validation(lib):
+    assert lib.attn_debug_set_fault(5, 0) == binding.ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_set_fault(0, 0) == binding.ATTN_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.fwd(x, x, x)

@@ -1,0 +1,102 @@
+"""GPU checks of the FP8 path: the quantisation kernel against the oracle's
+per-block e4m3 quantiser, and FP8 attention against the fp64 oracle on
+Gaussian inputs with outliers (with and without Hadamard rotation)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from io_aware_attention_02_b200 import inputs
+from oracle import attention as A
+from oracle import fp8 as F
+from parity_util import FP8_RMSE, errors
+
+pytestmark = pytest.mark.gpu
+
+
+def _x(B, H, N, d, seed, outliers=True):
+    return inputs.qkv(B, H, N, d, seed=seed, outliers=outliers)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [128, 300, 1024])
+def test_quant_plain_bit_exact(lib, d, N):
+    x = _x(2, 3, N, d, seed=N)[0]
+    codes, desc = lib.quant_fp8(x.cuda())
+    torch.cuda.synchronize()
+    c_ref, d_ref, _ = F.quantize_blocks(x.double().numpy())
+    np.testing.assert_array_equal(desc.cpu().numpy(), d_ref)
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("signed", [False, True])
+def test_quant_hadamard_close(lib, d, signed):
+    """With rotation the kernel's fp32 butterflies round differently from the
+    oracle's fp64 product: scales agree to fp32 rounding, codes agree except
+    where the value sits next to a rounding boundary (then one step apart)."""
+    x = _x(1, 4, 640, d, seed=7)[1]
+    signs = inputs.hadamard_signs(d, seed=3) if signed else None
+    codes, desc = lib.quant_fp8(x.cuda(), hadamard=True,
+                                signs=torch.from_numpy(signs) if signed else None)
+    torch.cuda.synchronize()
+    c_ref, d_ref, y = F.quantize_blocks(x.double().numpy(), True, signs)
+    np.testing.assert_allclose(desc.cpu().numpy(), d_ref, rtol=2e-6)
+    c = codes.cpu().numpy()
+    diff = c != c_ref
+    assert diff.mean() < 2e-3, diff.mean()
+    # where they differ both decode within one e4m3 step of y / s
+    vals = F.e4m3_decode(c)
+    s = np.repeat(d_ref.astype(np.float64), 128, axis=2)[:, :, :640, None]
+    t = y / s
+    step = np.maximum(np.abs(t) * 2.0 ** -3, 2.0 ** -9)
+    assert np.all(np.abs(vals[diff] - t[diff]) <= step[diff])
+
+
+def _fp8_attention(lib, q, k, v, causal, hadamard, signs=None):
+    sg = torch.from_numpy(signs) if signs is not None else None
+    q8, qd = lib.quant_fp8(q.cuda(), hadamard=hadamard, signs=sg)
+    k8, kd = lib.quant_fp8(k.cuda(), hadamard=hadamard, signs=sg)
+    v8, vd = lib.quant_fp8(v.cuda())
+    o, lse = lib.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=causal)
+    torch.cuda.synchronize()
+    return o, lse, (q8, k8, v8, qd, kd, vd)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hadamard", [False, True])
+@pytest.mark.parametrize("N", [128, 520])
+def test_fp8_attention_vs_fp64_oracle(lib, causal, hadamard, N):
+    q, k, v = _x(1, 4, N, 128, seed=30 + N)
+    signs = inputs.hadamard_signs(128, seed=1)
+    o, lse, packed = _fp8_attention(lib, q, k, v, causal, hadamard, signs)
+    scale = 1 / math.sqrt(128)
+    o_ref, l_ref = A.attention(q, k, v, scale, causal)
+    err = errors(o.cpu(), lse.cpu(), o_ref, l_ref)
+    assert err["rmse"] <= FP8_RMSE, err
+    # tighter: exact attention on the dequantised operands isolates the
+    # kernel's own arithmetic (P rounded to e4m3, fp32 accumulation)
+    q8, k8, v8, qd, kd, vd = (t.cpu().numpy() for t in packed)
+    qq = F.dequantize_blocks(q8, qd)
+    kk = F.dequantize_blocks(k8, kd)
+    vv = F.dequantize_blocks(v8, vd)
+    o_q, l_q = A.attention(qq, kk, vv, scale, causal)
+    err_q = errors(o.cpu(), lse.cpu(), o_q, l_q)
+    assert err_q["rmse"] <= 1.5e-2 and err_q["lse_max_abs"] <= 5e-3, err_q
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_headline_shape_sampled(lib, causal):
+    """B=4, H=16, N=8192, d=128 with outliers; Hadamard on; sampled rows."""
+    q, k, v = _x(4, 16, 8192, 128, seed=0)
+    signs = inputs.hadamard_signs(128, seed=0)
+    o, lse, _ = _fp8_attention(lib, q, k, v, causal, True, signs)
+    rows = inputs.sample_rows(8192, 32, seed=5)
+    heads = [(0, 0), (1, 5), (3, 15)]
+    scale = 1 / math.sqrt(128)
+    for b, h in heads:
+        o_ref, l_ref = A.attention_head(q[b, h], k[b, h], v[b, h], scale, causal, rows)
+        err = errors(o[b, h][rows].cpu(), lse[b, h][rows].cpu(), o_ref, l_ref)
+        assert err["rmse"] <= FP8_RMSE, (b, h, err)
