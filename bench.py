@@ -1,0 +1,401 @@
+#!/usr/bin/env python3
+"""Attention forward throughput on B200: one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one attention forward pass (attn_fwd through the C ABI) over the
+headline workload: B=4, H=16, N=8192, d=128, bf16, non-causal, seeded N(0,1)
+inputs.  ``value`` is TFLOP/s (4*B*H*N^2*d per step, halved for causal) over
+all ranks, with the inputs resident in HBM; ``e2e`` is the same metric when
+every step copies Q, K, V from pinned host memory and reads O and LSE back.
+The same line carries the causal and FP8 variants, the roofline of the
+kernel, clock samples taken during the timed region and (rank 0, one GPU) the
+CPU oracle timed on a bounded sample of the same workload.
+
+``--impl reference`` times the CPU oracle alone (fp64 definition, numpy) on a
+bounded sample of the workload and prints its line in the same metric.
+
+Multi-GPU (torchrun): every rank runs the same per-rank workload on its own
+GPU with no data exchange (weak scaling); the timed region is bracketed by a
+barrier and device synchronisation and the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from io_aware_attention_02_b200 import inputs  # noqa: E402
+
+WORKLOAD = dict(B=4, H=16, N=8192, d=128)
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_FP8_TFLOPS = 4500.0
+FALLBACK_BF16_TFLOPS = 1590.0
+METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16/FP8 tensor peak"
+
+# DRAM bytes per launch of the bf16 d=128 non-causal kernel on the workload
+# above, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
+# (profiles/attn_fwd_bf16_d128_B4H16N8192.md), keyed by the sha256 of the
+# kernel source it was measured on: reported only while the source is unchanged.
+TRAFFIC = {}
+
+
+def flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("fwd_sm100.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "io_aware_attention_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"bf16_tflops": FALLBACK_BF16_TFLOPS, "hbm_gbs": 6650.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 100):
+        self.index, self.period_ms, self.proc = index, period_ms, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world):
+    """Device time of `steps` calls of fn (ms), max over ranks."""
+    for _ in range(warmup):
+        fn()
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(s.elapsed_time(e), world)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (rank 0, one GPU only)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(q, k, v, causal, budget_s=15.0, gpu_out=None):
+    """Time the fp64 oracle on sampled query rows of a few heads.
+
+    Rows per head are chosen so that the work takes roughly `budget_s`.
+    Returns the cpu_baseline dict (value in TFLOP/s, same convention as the
+    GPU figure, counted on the rows computed).
+    """
+    from oracle import attention as A
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = len(os.sched_getaffinity(0))
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    heads = [(0, 0), (B - 1, H - 1), (B // 2, H // 2), (1 % B, 3 % H)]
+    # calibrate on 64 rows of one head
+    rows = inputs.sample_rows(N, 64, seed=11)
+    t0 = time.perf_counter()
+    A.attention_head(q[0, 0], k[0, 0], v[0, 0], scale, causal, rows)
+    per_row = (time.perf_counter() - t0) / len(rows)
+    n_rows = int(max(64, min(N, budget_s / max(per_row, 1e-9) / len(heads))))
+    rows = inputs.sample_rows(N, n_rows, seed=12)
+    errs = []
+    t0 = time.perf_counter()
+    for b, h in heads:
+        o, l = A.attention_head(q[b, h], k[b, h], v[b, h], scale, causal, rows)
+        if gpu_out is not None:
+            og = gpu_out[0][b, h][rows].double().cpu().numpy()
+            lg = gpu_out[1][b, h][rows].double().cpu().numpy()
+            errs.append((np.abs(og - o).max(), np.mean((og - o) ** 2), np.abs(lg - l).max()))
+    dt = time.perf_counter() - t0
+    # flops of the rows computed: 4*N*d per row (non-causal), halved for causal
+    # exactly as the throughput convention does
+    f = len(heads) * len(rows) * 4.0 * N * d / (2 if causal else 1)
+    out = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+           "sample": f"{len(rows)} query rows x {len(heads)} heads of B={B},H={H},N={N},d={d} "
+                     f"{'causal' if causal else 'non-causal'} (numpy fp64, full keys)",
+           "seconds": dt}
+    if errs:
+        e = np.array(errs)
+        out["parity_sample"] = {"max_abs_dO": float(e[:, 0].max()),
+                                "rmse_dO": float(math.sqrt(e[:, 1].mean())),
+                                "max_abs_dLSE": float(e[:, 2].max())}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    W = WORKLOAD
+    q, k, v = inputs.qkv(W["B"], W["H"], W["N"], W["d"], seed=0)
+    per_step = []
+    cb = None
+    # each step is a bounded sample, sized so that the whole run stays within
+    # about --ref-total seconds of CPU work
+    budget = max(0.05, min(args.ref_budget, args.ref_total / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(q, k, v, False, budget_s=budget)
+    for _ in range(args.steps):
+        cb = oracle_sample(q, k, v, False, budget_s=budget)
+        per_step.append(cb["seconds"])
+    val = cb["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * statistics.mean(per_step), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "B=4,H=16,N=8192,d=128 bf16 inputs, non-causal", **W,
+                       "causal": False},
+            "cpu_baseline": {k2: cb[k2] for k2 in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from io_aware_attention_02_b200 import binding
+    binding.load()
+    W = WORKLOAD
+    B, H, N, d = W["B"], W["H"], W["N"], W["d"]
+    dev = torch.device("cuda", local)
+    q, k, v = inputs.qkv(B, H, N, d, seed=rank)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    f_nc = flops(B, H, N, d, False)
+
+    def step():
+        binding.fwd(qd, kd, vd, causal=False, out=o, lse=lse)
+
+    with ClockSampler(local) as clk:
+        ms = timed(step, args.steps, args.warmup, world)
+    ms_step = ms / args.steps
+    value = world * f_nc / (ms_step * 1e-3) / 1e12
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} at {where}")
+
+    # causal variant, same shape
+    def step_c():
+        binding.fwd(qd, kd, vd, causal=True, out=o, lse=lse)
+    ms_c = timed(step_c, max(3, args.steps // 2), args.warmup, world) / max(3, args.steps // 2)
+    tf_c = flops(B, H, N, d, True) / (ms_c * 1e-3) / 1e12
+
+    # FP8 variant: outlier inputs, Hadamard rotation of Q and K, 128 x d block scales
+    qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank, outliers=True))
+    signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
+    q8, qs = binding.quant_fp8(qo, hadamard=True, signs=signs)
+    k8, ks = binding.quant_fp8(ko, hadamard=True, signs=signs)
+    v8, vs = binding.quant_fp8(vo)
+    o8 = torch.empty_like(qo)
+
+    def step_fp8():
+        binding.fwd_fp8(q8, k8, v8, qs, ks, vs, causal=False, out=o8, lse=lse)
+    n8 = max(3, args.steps // 2)
+    ms_8 = timed(step_fp8, n8, args.warmup, world) / n8
+
+    def step_quant():
+        binding.quant_fp8(qo, hadamard=True, signs=signs, out=q8, descale=qs)
+        binding.quant_fp8(ko, hadamard=True, signs=signs, out=k8, descale=ks)
+        binding.quant_fp8(vo, out=v8, descale=vs)
+    ms_q = timed(step_quant, n8, args.warmup, world) / n8
+    tf_8 = f_nc / (ms_8 * 1e-3) / 1e12
+
+    # e2e: pinned host inputs in, O and LSE out, every step
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lh = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def step_e2e():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        binding.fwd(qd, kd, vd, causal=False, out=o, lse=lse)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+    n_e = max(3, args.steps // 4)
+    ms_e = timed(step_e2e, n_e, min(args.warmup, 3), world) / n_e
+    e2e_val = world * f_nc / (ms_e * 1e-3) / 1e12
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = o.numel() * o.element_size() + lse.numel() * 4
+
+    peaks, src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    achieved = f_nc / (ms_step * 1e-3) / 1e12
+    khash = kernel_source_hash()
+    traffic = TRAFFIC.get(khash)
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) fp32 rounded to bf16",
+        "config": {"workload": "B=4,H=16,N=8192,d=128 bf16 non-causal", **W, "causal": False,
+                   "parallelism": f"replicas x{world} (independent batches, no exchange)",
+                   "l2": "inputs 384 MiB + output 128 MiB per step exceed the 126 MB L2; no flush"},
+        "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{src} bf16_tflops (burst cuBLAS 8192^3)",
+                     "algorithmic_flops_per_launch": f_nc, "kernel_source": khash},
+        "variants": {
+            "bf16_causal": {"tflops": tf_c, "ms": ms_c,
+                            "pct_of_spec_bf16_peak": 100 * tf_c / SPEC_BF16_TFLOPS},
+            "fp8_e4m3_hadamard_noncausal": {
+                "tflops": tf_8, "ms": ms_8, "pct_of_spec_fp8_peak": 100 * tf_8 / SPEC_FP8_TFLOPS,
+                "quant_ms_qkv": ms_q,
+                "tflops_incl_quant": f_nc / ((ms_8 + ms_q) * 1e-3) / 1e12,
+                "inputs": "N(0,1) with 0.1% entries replaced by N(0,10^2)"},
+        },
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        # o / lse hold the last e2e step's result for these same inputs
+        line["cpu_baseline"] = oracle_sample(q, k, v, False, budget_s=args.ref_budget,
+                                             gpu_out=(o.cpu(), lse.cpu()))
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=600)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-budget", type=float, default=15.0,
+                    help="seconds of CPU work per oracle sample")
+    ap.add_argument("--ref-total", type=float, default=150.0,
+                    help="seconds of CPU work for the whole reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the CPU oracle: rank 0 alone works, other ranks exit without work
+        run_reference(args, 1, int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
