@@ -131,6 +131,32 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
  */
 attn_status_t attn_last_status(void* stream, int* where);
 
+/*
+ * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device
+ * memory.  The pages have no counterpart: it exists for callers such as a
+ * process whose device memory is owned by a pool allocator or another
+ * runtime, or code that must not trigger cudaMalloc (whose first-use
+ * allocation attn_fwd performs for its status word) at a point where
+ * allocation is forbidden.
+ *   Arguments, layout, validation, results and error codes are those of
+ *   attn_fwd.  The only scratch the kernel needs -- the 16-byte record its
+ *   bounded waits write on a timeout -- lives in a static 256-byte device
+ *   array inside the library instead of memory the library allocates.  That
+ *   need does not grow with B, H, N or d, so no size exceeds the 256-byte
+ *   maximum; every GPU that loads the library holds the array until exit.
+ *   This entry point calls no cudaMalloc, cudaFree or allocating routine.
+ *   Its first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call clears the record on `stream` before its launch.  All calls
+ *   share the one array, so calls whose kernels overlap on the GPU (on
+ *   different streams) race on it.  A wait that runs out is recorded in that
+ *   shared record only: attn_last_status() does not see it, and the outputs
+ *   of that call are undefined.
+ */
+attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int N, int d, float scale, int causal, int dtype,
+                               void* stream);
+
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t s);
 

@@ -29,6 +29,7 @@ SIGNATURES = {
     "attn_last_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_debug_set_fault": (_I, [_I, _I]),
+    "attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
 }
 
 
@@ -110,6 +111,28 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     code = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse) if return_lse else None,
                            B, H, N, d, scale, int(bool(causal)), dtype, _stream(q.device))
     _check("attn_fwd", code)
+    return o, (lse if return_lse else None)
+
+
+def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                scale: float | None = None, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None, return_lse: bool = True):
+    """Like :func:`fwd`, through ``attn_fwd_noalloc``: the library allocates
+    no device memory for this call (its scratch is a static device array).
+    The outputs here are still allocated by torch unless passed in."""
+    _check_qkv(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bf16 or all fp16")
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
+    code = load().attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                   _ptr(lse) if return_lse else None, B, H, N, d, scale,
+                                   int(bool(causal)), dtype, _stream(q.device))
+    _check("attn_fwd_noalloc", code)
     return o, (lse if return_lse else None)
 
 

@@ -272,3 +272,89 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of attn_fwd (see include/attn.h).  Its scratch, the
+// kernel's 16-byte status record, lives in this file-scope device array; host
+// code uses the array's device address from cudaGetSymbolAddress, never the
+// host-side name.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;
+constexpr size_t kNoAllocStatusBytes = 4 * sizeof(int);
+static_assert(kNoAllocStatusBytes <= kNoAllocScratchBytes, "status record must fit the scratch array");
+static __device__ __align__(256) int g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int)];
+
+struct NoAllocDevice {
+  int* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int sm_count = 0;
+};
+NoAllocDevice g_noalloc_dev[kMaxDevices];
+
+// Once per device, with that device current: look up the array's address.
+attn_status_t noalloc_device(NoAllocDevice** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocDevice& st = g_noalloc_dev[dev];
+  if (st.scratch == nullptr) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    int* ptr = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch) != cudaSuccess ||
+        ptr == nullptr)
+      return ATTN_ERR_CUDA;
+    st.sm_count = sms;
+    st.scratch = ptr;
+  }
+  *out = &st;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                          float* lse, int B, int H, int N, int d, float scale,
+                                          int causal, int dtype, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+
+  NoAllocDevice* st = nullptr;
+  if ((r = noalloc_device(&st)) != ATTN_OK) return r;
+
+  const int BH = B * H;
+  const CUtensorMapDataType dt =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  attn::FwdParams p{};
+  if ((r = make_map(&p.tm_q, q, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  p.o = o;
+  p.lse = lse;
+  p.status = st->scratch;
+  p.BH = BH;
+  p.N = N;
+  p.n_kv = (N + 127) / 128;
+  p.n_qpairs = (N + 255) / 256;
+  p.n_units = BH * p.n_qpairs;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = wait_limit_ns();
+  p.fault = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the record keeps the previous call's contents: it must start at zero
+  if (cudaMemsetAsync(st->scratch, 0, kNoAllocStatusBytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  if (dtype == ATTN_BF16)
+    return d == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
+                   : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
+  return d == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
+                 : launch_fwd_c<__half, 128>(p, grid, causal, s);
+}

@@ -29,7 +29,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted(["attn_fwd", "attn_quant_fp8", "attn_fwd_fp8", "attn_last_status",
-                                  "attn_status_string", "attn_debug_set_fault"])
+                                  "attn_status_string", "attn_debug_set_fault",
+                                  "attn_fwd_noalloc"])
 
 
 def test_library_exports_every_declared_symbol(lib):
