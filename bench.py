@@ -284,6 +284,13 @@ def run_ours(args, world, rank, local):
     if code != 0:
         raise RuntimeError(f"kernel status {code} at {where}")
 
+    if args.only == "main":
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                              "only": "main"}), flush=True)
+        return
+
     # causal variant, same shape
     def step_c():
         binding.fwd(qd, kd, vd, causal=True, out=o, lse=lse)
@@ -381,6 +388,8 @@ def main():
     ap.add_argument("--ref-total", type=float, default=150.0,
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "main"], default="all",
+                    help="main: time only the bf16 non-causal step (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
