@@ -20,8 +20,9 @@
 //     metodo" item 3; quantum-bit repost, first technical upgrade);
 //   * warp 1: one thread issues every tcgen05.mma -- S_t = Q_t K_j^T
 //     (SMEM x SMEM -> TMEM) and O_t += P_t V_j (P from TMEM, V from SMEM);
-//   * warps 2-5 / 6-9: softmax warpgroups, one per Q tile, one thread per
-//     query row.  While one group turns S into P the tensor core works on the
+//   * warps 4-7 / 8-11: softmax warpgroups, one per Q tile, one thread per
+//     query row (warps 2-3 idle; setmaxnreg moves their registers and those
+//     of warps 0-1 to the softmax warpgroups).  While one group turns S into P the tensor core works on the
 //     other tile: the ping-pong schedule of the quantum-bit repost
 //     ("ping-pong scheduling") carried over to tcgen05;
 //   * causal: key tiles entirely above the diagonal are never loaded or
@@ -100,7 +101,7 @@ struct FwdCfg {
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStages = (kTileBytes <= 16384) ? 8 : 4;
   static constexpr int kKeysPerMma = 32 / Elem<E>::kBytes;  // 32 bytes of K per tcgen05.mma
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;   // 3 warpgroups: TMA+MMA | softmax 0 | softmax 1
   static constexpr int kTmemCols = 512;                   // S0 | S1 | O0 | O1
   static constexpr int kColS = 0;                         // + t * 128
   static constexpr int kColO = 256;                       // + t * D
@@ -118,8 +119,108 @@ enum : int {
   kWherePFull = 5, kWhereSFull = 6, kWhereOFull = 7, kWhereDrain = 8
 };
 
+// ---------------------------------------------------------------------------
+// Softmax arithmetic helpers
+// ---------------------------------------------------------------------------
+
+// max of 128 values with 3-input max instructions, four independent chains.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float a[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+  for (int i = 4; i < 128; i += 8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 4 + k]);
+  }
+  return fmax3(fmaxf(a[0], a[1]), a[2], a[3]);
+}
+
+// 2^x for a pair on the FMA pipe (Cody-Waite style split, then a minimax
+// polynomial): j = round(x) through the 1.5*2^23 addition, f = x - j in
+// [-1/2, 1/2], 2^f ~ p(f), and 2^j added into the exponent field with one
+// shift-add.  x is clamped to >= -125 so the exponent arithmetic cannot wrap
+// (2^-125 is far below anything that survives the final division by l).
+// Coefficients: minimax relative-error fit of degree kDeg (Remez exchange),
+// produced by io_aware_attention_02_b200/fit_exp2_poly.py; max relative
+// error 7.5e-5 (degree 3) / 1.7e-3 (degree 2).
+template <int kDeg>
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+  const float2 r = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+  const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), x);
+  float2 p;
+  if constexpr (kDeg == 3) {
+    p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                   make_float2(0.2426111251115799f, 0.2426111251115799f));
+    p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  } else {
+    p = __ffma2_rn(make_float2(0.23842893540859222f, 0.23842893540859222f), f,
+                   make_float2(0.7034479975700378f, 0.7034479975700378f));
+    p = __ffma2_rn(p, f, make_float2(1.0004431009292603f, 1.0004431009292603f));
+  }
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float2 exp2_mufu2(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
+// Pairs i with (i % 8) < kPolyPairsPer8 take the polynomial path.
+constexpr int kPolyPairsPer8 = 1;
+
+// P = 2^(s*c - m) for one half (64 keys, h = 0 or 1) of a 128-key row:
+// packed to 16-bit pairs (or e4m3 quads, after the gain) and written over the
+// row's S columns in TMEM (32 columns per half at 16 bit, 16 at e4m3).
+// Returns the fp32 sum of the unrounded P of that half.
+template <bool kF8, typename T, bool kPoly>
+__device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, float c, float neg_m,
+                                               float pgain, uint32_t tS) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(neg_m, neg_m);
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  if constexpr (!kF8) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = 64 * h + 2 * i;
+      const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, nm2);
+      const float2 pr = (kPoly && (i % 8) < kPolyPairsPer8) ? exp2_poly2<3>(x) : exp2_mufu2(x);
+      acc[i & 1] = __fadd2_rn(acc[i & 1], pr);
+      pk[i] = pack2<T>(pr.x, pr.y);
+    }
+    tmem_st32(tS + 32 * h, pk);
+  } else {
+    const float2 g2 = make_float2(pgain, pgain);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int e = 64 * h + 4 * i;
+      const float2 x0 = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, nm2);
+      const float2 x1 = __ffma2_rn(make_float2(s[e + 2], s[e + 3]), c2, nm2);
+      const float2 p0 = (kPoly && (i % 4) < 1) ? exp2_poly2<2>(x0) : exp2_mufu2(x0);
+      const float2 p1 = (kPoly && (i % 4) < 2) ? exp2_poly2<2>(x1) : exp2_mufu2(x1);
+      acc[0] = __fadd2_rn(acc[0], p0);
+      acc[1] = __fadd2_rn(acc[1], p1);
+      const float2 g0 = __fmul2_rn(p0, g2);
+      const float2 g1 = __fmul2_rn(p1, g2);
+      pk[i] = pack4_e4m3(g0.x, g0.y, g1.x, g1.y);
+    }
+    tmem_st16(tS + 16 * h, pk);
+  }
+  const float2 a = __fadd2_rn(acc[0], acc[1]);
+  return a.x + a.y;
+}
+
+constexpr int kRegsLow = 104;    // TMA + MMA warpgroup
+constexpr int kRegsHigh = 200;  // each softmax warpgroup
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch pool");
+
 template <typename E, int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using Cfg = FwdCfg<E, D>;
   using T = typename Elem<E>::Out;
   constexpr bool kF8 = Elem<E>::kF8;
@@ -133,12 +234,12 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* s_full = bars + 2;       // [2]
-  uint64_t* p_full = bars + 4;       // [2]
-  uint64_t* o_full = bars + 6;       // [2]
-  uint64_t* drain = bars + 8;
-  uint64_t* kv_full = bars + 9;      // [S]
-  uint64_t* kv_empty = bars + 9 + S; // [S]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * S);
+  uint64_t* p_full = bars + 4;       // [2 tiles][2 key halves]
+  uint64_t* o_full = bars + 8;       // [2]
+  uint64_t* drain = bars + 10;
+  uint64_t* kv_full = bars + 11;     // [S]
+  uint64_t* kv_empty = bars + 11 + S; // [S]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11 + 2 * S);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -149,7 +250,8 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
     mbar_init(q_empty, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, 128);
+      mbar_init(p_full + 2 * t, 128);
+      mbar_init(p_full + 2 * t + 1, 128);
       mbar_init(o_full + t, 1);
     }
     mbar_init(drain, 1);
@@ -172,6 +274,13 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
   const int n_kv = p.n_kv;
   const unsigned long long lim = p.wait_limit_ns;
 
+  // Register split (setmaxnreg acts per warpgroup): the TMA/MMA warpgroup
+  // gives registers to the two softmax warpgroups.  128*104 + 256*200 =
+  // 64512 = 384 threads * 168 registers, the launch allocation.  Each
+  // setmaxnreg sits inside its role's branch, so no code after a control-flow
+  // merge is held to the lower count.
+  if (warp < 4) {
+  reg_dealloc<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -226,41 +335,52 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
       constexpr uint32_t fmt = Elem<E>::kFmt;
       constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, 0, 128, 128);
       constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 0, 1, 128, D);
-      const uint32_t sQ_addr = smem_u32(sQ);
-      const uint32_t sKV_addr = smem_u32(sKV);
       uint32_t kv_iter = 0, unit_iter = 0;
       uint32_t p_cnt[2] = {0, 0};
       bool ok = true;
 
+      // Descriptors are built once and advanced by adding (byte offset >> 4)
+      // to their start-address field (addresses stay below 256 KiB, so the
+      // 14-bit field never carries).
+      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(sKV), Cfg::kChunkBytes, 1024);
+
       auto issue_s = [&](int t, uint32_t kstage) {
-        const uint32_t a0 = sQ_addr + t * Cfg::kTileBytes;
-        const uint32_t b0 = sKV_addr + kstage * Cfg::kTileBytes;
+        const uint64_t a0 = dQ + static_cast<uint64_t>((t * Cfg::kTileBytes) >> 4);
+        const uint64_t b0 = dK + static_cast<uint64_t>((kstage * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
           // K-major, 128-byte swizzle: each product consumes 32 bytes of the
           // head dim; four of them span one 128-byte chunk row.
-          const uint32_t off = (kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::kColS + t * 128, smem_desc_sw128(a0 + off, 16, 1024),
-                 smem_desc_sw128(b0 + off, 16, 1024), idesc_s, kk > 0, kF8);
+          const uint32_t off = ((kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + Cfg::kColS + t * 128, a0 + off, b0 + off, idesc_s, kk > 0, kF8);
         }
       };
-      auto issue_pv = [&](int t, uint32_t vstage, bool acc) {
-        const uint32_t b0 = sKV_addr + vstage * Cfg::kTileBytes;
+      // One half (64 keys) of O_t += P_t V_j.
+      auto issue_pv_half = [&](int t, uint32_t vstage, int h, bool acc) {
+        const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);
+        constexpr int kSteps = 64 / Cfg::kKeysPerMma;
 #pragma unroll
-        for (int kk = 0; kk < 128 / Cfg::kKeysPerMma; ++kk) {
+        for (int kk = h * kSteps; kk < (h + 1) * kSteps; ++kk) {
           // P_t: 128 rows x 128 keys packed in TMEM (32 bytes = 8 columns per
           // product).  V_j: MN-major (head dim contiguous), kKeysPerMma keys
           // = kKeysPerMma rows of 128 bytes per product.
           mma_ts(tmem + Cfg::kColO + t * D, tmem + Cfg::kColS + t * 128 + kk * 8,
-                 smem_desc_sw128(b0 + kk * Cfg::kKeysPerMma * 128, Cfg::kChunkBytes, 1024), idesc_o,
-                 (acc || kk > 0) ? 1u : 0u, kF8);
+                 b0 + ((kk * Cfg::kKeysPerMma * 128) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
         }
       };
-      auto wait_p = [&](int t) -> bool {
-        bool r = mbar_wait(p_full + t, p_cnt[t] & 1, p.status, abort_flag, kWherePFull, lim);
+      // O_t += P_t V_j as soon as each half of P_t is in TMEM: the first
+      // half's products run while the softmax still computes the second.
+      auto pv = [&](int t, uint32_t vstage, bool acc) -> bool {
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(p_full + 2 * t + h, p_cnt[t] & 1, p.status, abort_flag, kWherePFull, lim))
+            return false;
+          tc_fence_after();
+          issue_pv_half(t, vstage, h, acc);
+        }
         ++p_cnt[t];
-        tc_fence_after();
-        return r;
+        return true;
       };
       auto wait_kv = [&](uint32_t idx) -> bool {
         bool r = mbar_wait(kv_full + (idx % S), (idx / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
@@ -291,17 +411,14 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
           if (!(ok = wait_kv(ik))) break;
           if (!(ok = wait_kv(iv))) break;
           if (j < n0) {
-            if (!(ok = wait_p(0))) break;
-            issue_pv(0, iv % S, j - 1 > 0);
+            if (!(ok = pv(0, iv % S, j - 1 > 0))) break;
             issue_s(0, ik % S);
             mma_commit(s_full + 0);
           } else if (j == n0) {
-            if (!(ok = wait_p(0))) break;
-            issue_pv(0, iv % S, j - 1 > 0);
+            if (!(ok = pv(0, iv % S, j - 1 > 0))) break;
             mma_commit(o_full + 0);
           }
-          if (!(ok = wait_p(1))) break;
-          issue_pv(1, iv % S, j - 1 > 0);
+          if (!(ok = pv(1, iv % S, j - 1 > 0))) break;
           mma_commit(kv_empty + (iv % S));
           issue_s(1, ik % S);
           mma_commit(s_full + 1);
@@ -311,12 +428,10 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
         const uint32_t iv = base + 2 * (n1 - 1) + 1;
         if (!(ok = wait_kv(iv))) break;
         if (n0 == n1) {
-          if (!(ok = wait_p(0))) break;
-          issue_pv(0, iv % S, n1 - 1 > 0);
+          if (!(ok = pv(0, iv % S, n1 - 1 > 0))) break;
           mma_commit(o_full + 0);
         }
-        if (!(ok = wait_p(1))) break;
-        issue_pv(1, iv % S, n1 - 1 > 0);
+        if (!(ok = pv(1, iv % S, n1 - 1 > 0))) break;
         mma_commit(o_full + 1);
         mma_commit(kv_empty + (iv % S));
         mma_commit(q_empty);
@@ -330,9 +445,11 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
       }
     }
     __syncwarp();
+  }
   } else {
+    reg_alloc<kRegsHigh>();
     // -------------------------------------------------------------- softmax
-    const int t = (warp - 2) >> 2;                 // Q tile (slot) 0 or 1
+    const int t = (warp - 4) >> 2;                 // Q tile (slot) 0 or 1
     const int quarter = warp & 3;                  // TMEM lane quarter this warp may access
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -398,10 +515,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
           for (int i = 0; i < 128; ++i)
             if (key0 + i > lim_key) s[i] = -INFINITY;
         }
-        float mx = s[0];
-#pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-        mx *= c;
+        const float mx = row_max128(s) * c;
         // Lazy max: raise m only when the tile max exceeds it by more than
         // kLazy (log2 units); then alpha = 2^(m_old - m_new), 0 on the first
         // tile.  The final division by l makes the stale max exact.
@@ -410,39 +524,9 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
           alpha = ex2_approx(m - mx);
           m = mx;
         }
-        const float neg_m = -m;
-        float sum = 0.f;
-        if constexpr (!kF8) {
-          // two halves of 64 keys -> 32 packed columns each, so that only
-          // half of P is live in registers at a time
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = ex2_approx(fmaf(s[64 * hf + 2 * i], c, neg_m));
-              const float p1 = ex2_approx(fmaf(s[64 * hf + 2 * i + 1], c, neg_m));
-              sum += p0 + p1;
-              pk[i] = pack2<T>(p0, p1);
-            }
-            tmem_st32(tS + 32 * hf, pk);
-          }
-        } else {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2_approx(fmaf(s[4 * i], c, neg_m));
-            const float p1 = ex2_approx(fmaf(s[4 * i + 1], c, neg_m));
-            const float p2 = ex2_approx(fmaf(s[4 * i + 2], c, neg_m));
-            const float p3 = ex2_approx(fmaf(s[4 * i + 3], c, neg_m));
-            sum += (p0 + p1) + (p2 + p3);
-            pk[i] = pack4_e4m3(p0 * pgain, p1 * pgain, p2 * pgain, p3 * pgain);
-          }
-          tmem_st32(tS, pk);
-        }
-        l = l * alpha + sum;
-        // Rescale O_t when some row of this warp raised its max.  The PV
-        // product of the previous key tile has completed: S_t(j) was
+        // Rescale O_t when some row of this warp raised its max, before the
+        // first half of P is published (its PV product accumulates into O_t).
+        // The PV product of the previous key tile has completed: S_t(j) was
         // committed after it.
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
@@ -455,9 +539,20 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_sm100_kernel(const __grid_con
             tmem_st32(tO + cc * 32, r);
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + t);
+        // P in two halves of 64 keys, each published as soon as it is in
+        // TMEM.  Masked tiles hold -inf scores, which only the MUFU path maps
+        // to an exact 0; unmasked tiles may send part of their exp2 work to
+        // the FMA pipe.
+        float sum = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          sum += need_mask ? exp_pack_half<kF8, T, false>(s, h, c, -m, pgain, tS)
+                           : exp_pack_half<kF8, T, true>(s, h, c, -m, pgain, tS);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full + 2 * t + h);
+        }
+        l = l * alpha + sum;
       }
       if (!ok) break;
 
