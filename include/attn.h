@@ -66,8 +66,7 @@ typedef enum {
  *   q, k, v : [B][H][N][d] bf16 or fp16 (per `dtype`), read only.
  *   o       : [B][H][N][d] same dtype, written.
  *   lse     : [B][H][N] fp32, written; may be NULL (then not written).
- *   B, H, N : >= 1, B*H*N < 2^31.   d : 64 or 128 (256: ATTN_ERR_UNSUPPORTED
- *             in this build).
+ *   B, H, N : >= 1, B*H*N < 2^31.   d : 64, 128 or 256.
  *   scale   : finite and > 0 (usually 1/sqrt(d)).
  *   causal  : 0 or 1 (key j visible to query i iff j <= i).
  * Rounding: scores, statistics and accumulation are fp32; P is rounded to
@@ -139,7 +138,8 @@ attn_status_t attn_last_status(void* stream, int* where);
  * allocation attn_fwd performs for its status word) at a point where
  * allocation is forbidden.
  *   Arguments, layout, validation, results and error codes are those of
- *   attn_fwd.  The only scratch the kernel needs -- the 16-byte record its
+ *   attn_fwd, for head dims 64 and 128 (256 returns ATTN_ERR_UNSUPPORTED
+ *   here).  The only scratch the kernel needs -- the 16-byte record its
  *   bounded waits write on a timeout -- lives in a static 256-byte device
  *   array inside the library instead of memory the library allocates.  That
  *   need does not grow with B, H, N or d, so no size exceeds the 256-byte

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "quant_fp8.cuh"
 
@@ -120,6 +121,26 @@ attn_status_t launch_fwd_c(const attn::FwdParams& p, int grid, int causal, cudaS
   return causal ? launch_fwd<E, D, true>(p, grid, s) : launch_fwd<E, D, false>(p, grid, s);
 }
 
+// Head dim 256: one 128-row Q tile per work unit (n_qpairs then counts
+// 128-row tiles).
+template <typename E, bool CAUSAL>
+attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream) {
+  using Cfg = attn::Fwd256Cfg;
+  auto kern = attn::attn_fwd_sm100_d256_kernel<E, CAUSAL>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_done = true;
+  }
+  p.n_qpairs = (p.N + 127) / 128;
+  p.n_units = p.BH * p.n_qpairs;
+  const int grid = p.n_units < sm_count ? p.n_units : sm_count;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // Fills the fields shared by the 16-bit and FP8 launches.
 attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void* o, int BH, int N,
                           float scale) {
@@ -188,7 +209,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   attn_status_t r = common_checks(B, H, N, scale, causal);
   if (r != ATTN_OK) return r;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
@@ -206,6 +227,13 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   fill_common(&p, st, lse, o, BH, N, scale);
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256) {
+    if (dtype == ATTN_BF16)
+      return causal ? launch_fwd256<__nv_bfloat16, true>(p, st->sm_count, s)
+                    : launch_fwd256<__nv_bfloat16, false>(p, st->sm_count, s);
+    return causal ? launch_fwd256<__half, true>(p, st->sm_count, s)
+                  : launch_fwd256<__half, false>(p, st->sm_count, s);
+  }
   if (dtype == ATTN_BF16)
     return d == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);

@@ -22,7 +22,7 @@ def test_small_workload_full(lib):
     assert code == 0, where
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 100, 127, 128, 129, 255, 256, 257, 500, 1000])
 def test_ragged_and_multi_tile(lib, d, causal, N):
@@ -30,18 +30,19 @@ def test_ragged_and_multi_tile(lib, d, causal, N):
     assert_bf16_ok(err, (N, d, causal))
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_fp16(lib, d, causal):
     err, _ = run_and_compare(lib, 2, 3, 300, d, causal, dtype=torch.float16, seed=5)
     assert_bf16_ok(err, ("fp16", d, causal))
 
 
+@pytest.mark.parametrize("d", [64, 256])
 @pytest.mark.parametrize("causal", [False, True])
-def test_persistent_grid_wraps(lib, causal):
-    """B*H*ceil(N/256) > number of SMs, so each CTA takes several work units."""
-    err, _ = run_and_compare(lib, 2, 96, 512, 64, causal, seed=3)
-    assert_bf16_ok(err, ("wrap", causal))
+def test_persistent_grid_wraps(lib, causal, d):
+    """More work units than SMs, so each CTA takes several of them."""
+    err, _ = run_and_compare(lib, 2, 96, 512, d, causal, seed=3)
+    assert_bf16_ok(err, ("wrap", causal, d))
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -53,7 +54,8 @@ def test_headline_shape_sampled_rows(lib, causal):
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
 
 
-@pytest.mark.parametrize("N,d", [(512, 64), (2048, 128), (16384, 64), (16384, 128)])
+@pytest.mark.parametrize("N,d", [(512, 64), (2048, 128), (16384, 64), (16384, 128), (1024, 256),
+                                 (16384, 256)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_sequence_sweep_sampled(lib, N, d, causal):
     """Sweep shapes: total tokens B*N = 16K, H = 16; sampled heads and rows."""
