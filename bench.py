@@ -310,6 +310,10 @@ def run_ours(args, world, rank, local):
     n8 = max(3, args.steps // 2)
     ms_8 = timed(step_fp8, n8, args.warmup, world) / n8
 
+    def step_fp8_vt():
+        binding.fwd_fp8(q8, k8, v8, qs, ks, vs, causal=False, v_transpose=True, out=o8, lse=lse)
+    ms_8t = timed(step_fp8_vt, n8, args.warmup, world) / n8
+
     def step_quant():
         binding.quant_fp8(qo, hadamard=True, signs=signs, out=q8, descale=qs)
         binding.quant_fp8(ko, hadamard=True, signs=signs, out=k8, descale=ks)
@@ -363,6 +367,7 @@ def run_ours(args, world, rank, local):
                 "tflops": tf_8, "ms": ms_8, "pct_of_spec_fp8_peak": 100 * tf_8 / SPEC_FP8_TFLOPS,
                 "quant_ms_qkv": ms_q,
                 "tflops_incl_quant": f_nc / ((ms_8 + ms_q) * 1e-3) / 1e12,
+                "tflops_v_transpose": f_nc / (ms_8t * 1e-3) / 1e12,
                 "inputs": "N(0,1) with 0.1% entries replaced by N(0,10^2)"},
         },
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

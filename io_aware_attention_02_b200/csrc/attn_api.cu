@@ -101,10 +101,10 @@ attn_status_t common_checks(int B, int H, int N, float scale, int causal) {
   return ATTN_OK;
 }
 
-template <typename E, int D, bool CAUSAL>
+template <typename E, int D, bool CAUSAL, bool VT = false>
 attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<E, D>;
-  auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL>;
+  auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL, VT>;
   static bool attr_done = false;  // per instance; set once per process
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
@@ -276,7 +276,6 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   if (v_transpose != 0 && v_transpose != 1) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (v_transpose != 0) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
   const uintptr_t a4 = reinterpret_cast<uintptr_t>(q_descale) | reinterpret_cast<uintptr_t>(k_descale) |
                        reinterpret_cast<uintptr_t>(v_descale) |
@@ -296,7 +295,11 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   p.v_desc = v_descale;
   fill_common(&p, st, lse, o, BH, N, scale);
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
-  return launch_fwd_c<__nv_fp8_e4m3, 128>(p, grid, causal, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (v_transpose)
+    return causal ? launch_fwd<__nv_fp8_e4m3, 128, true, true>(p, grid, s)
+                  : launch_fwd<__nv_fp8_e4m3, 128, false, true>(p, grid, s);
+  return launch_fwd_c<__nv_fp8_e4m3, 128>(p, grid, causal, s);
 }
 
 }  // extern "C"

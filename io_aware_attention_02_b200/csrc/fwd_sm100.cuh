@@ -105,11 +105,14 @@ struct FwdCfg {
   static constexpr int kTmemCols = 512;                   // S0 | S1 | O0 | O1
   static constexpr int kColS = 0;                         // + t * 128
   static constexpr int kColO = 256;                       // + t * D
-  // dynamic shared memory: [Q0 | Q1 | ring of kStages tiles | barriers]
+  // dynamic shared memory: [Q0 | Q1 | ring of kStages tiles | 2 transposed
+  // V tiles (FP8 only) | barriers]
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kBarBytes = 256;
+  static constexpr int kOffVt = kOffKV + kStages * kTileBytes;
+  static constexpr int kVtBytes = Elem<E>::kF8 ? 2 * kTileBytes : 0;
+  static constexpr int kOffBar = kOffVt + kVtBytes;
+  static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + 1 KiB alignment slack
 };
 
@@ -215,12 +218,59 @@ __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, flo
   return a.x + a.y;
 }
 
+// In-shared-memory transpose of one FP8 V tile (128 keys x 128 head-dim
+// bytes), from the TMA layout (MN-major for the P.V product: one 128-byte row
+// per key, 16-byte chunks swizzled by key % 8) to the K-major layout (one
+// 128-byte row per head-dim column, chunks swizzled by column % 8).  64
+// threads each move one 16 x 16 byte block with 16-byte loads and stores and
+// a register transpose of 4 x 4 byte blocks (byte permutes); block (kb, cb)
+// of thread t is kb = t % 8, cb = (t % 8 + t / 8) % 8, so that the 8 threads
+// of a quarter warp touch 8 distinct 16-byte bank groups on both sides.
+// This is the pages' V-tile transpose for FP8 (quantum-bit repost, FP8
+// paragraph: FP8 tensor cores want the reduction dim contiguous, so blocks of
+// V are transposed in place).
+__device__ __forceinline__ void transpose_v_tile_e4m3(const uint8_t* src, uint8_t* dst, int t) {
+  const int kb = t & 7;
+  const int cb = ((t & 7) + (t >> 3)) & 7;
+  uint32_t w[16][4];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int key = kb * 16 + r;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + key * 128 + ((cb ^ (key & 7)) << 4));
+    w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
+  }
+  // For each 4-column group q: rows c = 4q .. 4q+3 of the output, word g =
+  // bytes of column cb*16 + c for keys kb*16 + 4g .. 4g+3; stored at once so
+  // only 16 output words are live.
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t o[4][4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t a = w[4 * g][q], b = w[4 * g + 1][q], c = w[4 * g + 2][q], d = w[4 * g + 3][q];
+      const uint32_t t0 = __byte_perm(a, b, 0x5140), t1 = __byte_perm(a, b, 0x7362);
+      const uint32_t t2 = __byte_perm(c, d, 0x5140), t3 = __byte_perm(c, d, 0x7362);
+      o[0][g] = __byte_perm(t0, t2, 0x5410);
+      o[1][g] = __byte_perm(t0, t2, 0x7632);
+      o[2][g] = __byte_perm(t1, t3, 0x5410);
+      o[3][g] = __byte_perm(t1, t3, 0x7632);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int col = cb * 16 + 4 * q + k;
+      *reinterpret_cast<uint4*>(dst + col * 128 + ((kb ^ (col & 7)) << 4)) =
+          make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
+    }
+  }
+}
+
 constexpr int kRegsLow = 104;    // TMA + MMA warpgroup
 constexpr int kRegsHigh = 200;  // each softmax warpgroup
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch pool");
 
-template <typename E, int D, bool CAUSAL>
+template <typename E, int D, bool CAUSAL, bool VT = false>
 __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
+  static_assert(!VT || (Elem<E>::kF8 && D == 128), "V transpose is the FP8 d=128 path");
   using Cfg = FwdCfg<E, D>;
   using T = typename Elem<E>::Out;
   constexpr bool kF8 = Elem<E>::kF8;
@@ -239,7 +289,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
   uint64_t* drain = bars + 10;
   uint64_t* kv_full = bars + 11;     // [S]
   uint64_t* kv_empty = bars + 11 + S; // [S]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11 + 2 * S);
+  uint64_t* vt_full = bars + 11 + 2 * S;   // [2] transposed V tile ready (FP8, VT)
+  uint64_t* vt_empty = bars + 13 + 2 * S;  // [2] transposed V tile consumed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15 + 2 * S);
+  uint8_t* sVt = smem + Cfg::kOffVt;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -258,6 +311,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
     for (int s = 0; s < S; ++s) {
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(vt_full + b, 1);
+      mbar_init(vt_empty + b, 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -334,7 +391,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
     if (lane == 0) {
       constexpr uint32_t fmt = Elem<E>::kFmt;
       constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, 0, 128, 128);
-      constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 0, 1, 128, D);
+      // P.V with V MN-major straight from the TMA tile, or (VT) K-major from
+      // the transposed copy
+      constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 0, VT ? 0 : 1, 128, D);
       uint32_t kv_iter = 0, unit_iter = 0;
       uint32_t p_cnt[2] = {0, 0};
       bool ok = true;
@@ -344,7 +403,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       // 14-bit field never carries).
       const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t dV = smem_desc_sw128(smem_u32(sKV), Cfg::kChunkBytes, 1024);
+      const uint64_t dV = VT ? smem_desc_sw128(smem_u32(sVt), 16, 1024)
+                             : smem_desc_sw128(smem_u32(sKV), Cfg::kChunkBytes, 1024);
+      uint32_t v_cnt = 0;   // V tiles consumed (VT: selects the transposed buffer and phase)
 
       auto issue_s = [&](int t, uint32_t kstage) {
         const uint64_t a0 = dQ + static_cast<uint64_t>((t * Cfg::kTileBytes) >> 4);
@@ -359,15 +420,16 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       };
       // One half (64 keys) of O_t += P_t V_j.
       auto issue_pv_half = [&](int t, uint32_t vstage, int h, bool acc) {
-        const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);
+        const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);  // stage or Vt buffer
         constexpr int kSteps = 64 / Cfg::kKeysPerMma;
 #pragma unroll
         for (int kk = h * kSteps; kk < (h + 1) * kSteps; ++kk) {
           // P_t: 128 rows x 128 keys packed in TMEM (32 bytes = 8 columns per
           // product).  V_j: MN-major (head dim contiguous), kKeysPerMma keys
           // = kKeysPerMma rows of 128 bytes per product.
+          const uint32_t voff = VT ? ((kk * 32) >> 4) : ((kk * Cfg::kKeysPerMma * 128) >> 4);
           mma_ts(tmem + Cfg::kColO + t * D, tmem + Cfg::kColS + t * 128 + kk * 8,
-                 b0 + ((kk * Cfg::kKeysPerMma * 128) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
+                 b0 + voff, idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
         }
       };
       // O_t += P_t V_j as soon as each half of P_t is in TMEM: the first
@@ -386,6 +448,29 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         bool r = mbar_wait(kv_full + (idx % S), (idx / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
         tc_fence_after();
         return r;
+      };
+      // V_j for the P.V products: the ring stage itself, or (VT) the
+      // transposed copy; returns the value pv() takes as its V "stage".
+      auto wait_v = [&](uint32_t idx, bool& r) -> uint32_t {
+        if constexpr (VT) {
+          const uint32_t b = v_cnt & 1;
+          r = mbar_wait(vt_full + b, (v_cnt >> 1) & 1, p.status, abort_flag, kWhereKvFull, lim);
+          tc_fence_after();
+          return b;
+        } else {
+          r = wait_kv(idx);
+          return idx % S;
+        }
+      };
+      // Release V_j after both tiles' products: the ring stage (the
+      // transposer already released it under VT) or the transposed buffer.
+      auto release_v = [&](uint32_t vstage) {
+        if constexpr (VT) {
+          mma_commit(vt_empty + vstage);
+          ++v_cnt;
+        } else {
+          mma_commit(kv_empty + vstage);
+        }
       };
 
       for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
@@ -409,31 +494,33 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         for (int j = 1; j < n1 && ok; ++j) {
           const uint32_t ik = base + 2 * j, iv = base + 2 * (j - 1) + 1;
           if (!(ok = wait_kv(ik))) break;
-          if (!(ok = wait_kv(iv))) break;
+          const uint32_t vs = wait_v(iv, ok);
+          if (!ok) break;
           if (j < n0) {
-            if (!(ok = pv(0, iv % S, j - 1 > 0))) break;
+            if (!(ok = pv(0, vs, j - 1 > 0))) break;
             issue_s(0, ik % S);
             mma_commit(s_full + 0);
           } else if (j == n0) {
-            if (!(ok = pv(0, iv % S, j - 1 > 0))) break;
+            if (!(ok = pv(0, vs, j - 1 > 0))) break;
             mma_commit(o_full + 0);
           }
-          if (!(ok = pv(1, iv % S, j - 1 > 0))) break;
-          mma_commit(kv_empty + (iv % S));
+          if (!(ok = pv(1, vs, j - 1 > 0))) break;
+          release_v(vs);
           issue_s(1, ik % S);
           mma_commit(s_full + 1);
           mma_commit(kv_empty + (ik % S));
         }
         if (!ok) break;
         const uint32_t iv = base + 2 * (n1 - 1) + 1;
-        if (!(ok = wait_kv(iv))) break;
+        const uint32_t vs = wait_v(iv, ok);
+        if (!ok) break;
         if (n0 == n1) {
-          if (!(ok = pv(0, iv % S, n1 - 1 > 0))) break;
+          if (!(ok = pv(0, vs, n1 - 1 > 0))) break;
           mma_commit(o_full + 0);
         }
-        if (!(ok = pv(1, iv % S, n1 - 1 > 0))) break;
+        if (!(ok = pv(1, vs, n1 - 1 > 0))) break;
         mma_commit(o_full + 1);
-        mma_commit(kv_empty + (iv % S));
+        release_v(vs);
         mma_commit(q_empty);
         kv_iter += 2 * n1;
       }
@@ -445,6 +532,36 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       }
     }
     __syncwarp();
+  } else if (VT) {
+    // ---------------------------------------------------------- V transpose
+    // Warps 2-3: each V tile of the ring, in the order the MMA consumes
+    // them, into one of two K-major buffers; then release the ring stage.
+    const int tt = threadIdx.x - 64;              // 0..63
+    uint32_t kv_iter = 0, v_cnt = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
+      const int qr = unit % p.n_qpairs;
+      const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+      const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
+      for (int j = 0; j < n1; ++j, ++v_cnt) {
+        const uint32_t iv = kv_iter + 2 * j + 1;
+        const uint32_t b = v_cnt & 1;
+        bool w = mbar_wait(kv_full + (iv % S), (iv / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
+        w = w && mbar_wait(vt_empty + b, ((v_cnt >> 1) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
+        if (!__all_sync(0xffffffffu, w)) *abort_flag = 1;
+        named_bar_sync(3, 64);
+        if (*abort_flag) { ok = false; break; }
+        transpose_v_tile_e4m3(sKV + (iv % S) * Cfg::kTileBytes, sVt + b * Cfg::kTileBytes, tt);
+        // generic-proxy shared-memory writes, read next by the tensor core
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_bar_sync(3, 64);
+        if (tt == 0) {
+          mbar_arrive(kv_empty + (iv % S));
+          mbar_arrive(vt_full + b);
+        }
+      }
+      kv_iter += 2 * n1;
+    }
   }
   } else {
     reg_alloc<kRegsHigh>();

@@ -100,3 +100,24 @@ def test_fp8_headline_shape_sampled(lib, causal):
         o_ref, l_ref = A.attention_head(q[b, h], k[b, h], v[b, h], scale, causal, rows)
         err = errors(o[b, h][rows].cpu(), lse[b, h][rows].cpu(), o_ref, l_ref)
         assert err["rmse"] <= FP8_RMSE, (b, h, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 700, 2048])
+def test_v_transpose_matches_mn_major(lib, causal, N):
+    """The in-shared-memory V transpose feeds the same values to the tensor
+    core in K-major order: the output equals the MN-major path's."""
+    q, k, v = _x(2, 3, N, 128, seed=40 + N)
+    signs = inputs.hadamard_signs(128, seed=2)
+    sg = torch.from_numpy(signs)
+    q8, qd = lib.quant_fp8(q.cuda(), hadamard=True, signs=sg)
+    k8, kd = lib.quant_fp8(k.cuda(), hadamard=True, signs=sg)
+    v8, vd = lib.quant_fp8(v.cuda())
+    o0, l0 = lib.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=causal, v_transpose=False)
+    o1, l1 = lib.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=causal, v_transpose=True)
+    torch.cuda.synchronize()
+    assert lib.last_status()[0] == 0
+    # same products in the same order: bit-identical
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    o_ref, _ = A.attention(q, k, v, 1 / math.sqrt(128), causal)
+    assert errors(o1.cpu(), None, o_ref, None)["rmse"] <= FP8_RMSE
