@@ -132,17 +132,24 @@ class ClockSampler:
 # distributed plumbing
 # ---------------------------------------------------------------------------
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU: (world, rank, local rank) from the torchrun env.
+
+    The process group only carries barriers and the one-scalar max of the
+    timings: the per-rank workloads are independent (no data exchange).
+    """
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -154,12 +161,24 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank scalar over all ranks (the job time is the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank):
+    """Each rank draws its own batch (weak scaling: same per-rank work)."""
+    return rank
+
+
+def job_throughput(per_rank_flops, world, max_ms):
+    """Whole-job TFLOP/s: all ranks' work over the slowest rank's time."""
+    return world * per_rank_flops / (max_ms * 1e-3) / 1e12
 
 
 def timed(fn, steps, warmup, world):
@@ -267,7 +286,7 @@ def run_ours(args, world, rank, local):
     W = WORKLOAD
     B, H, N, d = W["B"], W["H"], W["N"], W["d"]
     dev = torch.device("cuda", local)
-    q, k, v = inputs.qkv(B, H, N, d, seed=rank)
+    q, k, v = inputs.qkv(B, H, N, d, seed=rank_seed(rank))
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     o = torch.empty_like(qd)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -279,7 +298,7 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         ms = timed(step, args.steps, args.warmup, world)
     ms_step = ms / args.steps
-    value = world * f_nc / (ms_step * 1e-3) / 1e12
+    value = job_throughput(f_nc, world, ms_step)
     code, where = binding.last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {code} at {where}")
@@ -298,7 +317,7 @@ def run_ours(args, world, rank, local):
     tf_c = flops(B, H, N, d, True) / (ms_c * 1e-3) / 1e12
 
     # FP8 variant: outlier inputs, Hadamard rotation of Q and K, 128 x d block scales
-    qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank, outliers=True))
+    qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank_seed(rank), outliers=True))
     signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
     q8, qs = binding.quant_fp8(qo, hadamard=True, signs=signs)
     k8, ks = binding.quant_fp8(ko, hadamard=True, signs=signs)
@@ -335,7 +354,7 @@ def run_ours(args, world, rank, local):
         lh.copy_(lse, non_blocking=True)
     n_e = max(3, args.steps // 4)
     ms_e = timed(step_e2e, n_e, min(args.warmup, 3), world) / n_e
-    e2e_val = world * f_nc / (ms_e * 1e-3) / 1e12
+    e2e_val = job_throughput(f_nc, world, ms_e)
     h2d = 3 * q.numel() * q.element_size()
     d2h = o.numel() * o.element_size() + lse.numel() * 4
 
@@ -382,6 +401,32 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """TFLOP/s of attn_fwd over the sequence sweep (total tokens B*N = 16K,
+    H = 16, d in {64, 128, 256}, causal and not) and the long-context case
+    (B=1, H=32, N=65536, d=128, causal); one JSON line per configuration."""
+    from io_aware_attention_02_b200 import binding
+    torch.cuda.set_device(0)
+    cases = [(16384 // n, 16, n, d, c) for d in (64, 128, 256) for n in (512, 1024, 2048, 4096, 8192, 16384)
+             for c in (False, True)]
+    cases.append((1, 32, 65536, 128, True))
+    for B, H, N, d, causal in cases:
+        g = torch.Generator(device="cuda").manual_seed(0)
+        q, k, v = (torch.randn(B, H, N, d, device="cuda", dtype=torch.bfloat16, generator=g) for _ in range(3))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+        steps = max(5, min(200, int(2e13 / flops(B, H, N, d, causal))))
+        ms = timed(lambda: binding.fwd(q, k, v, causal=causal, out=o, lse=lse), steps, 5, 1) / steps
+        tf = flops(B, H, N, d, causal) / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": True, "B": B, "H": H, "N": N, "d": d, "causal": causal, "ms": ms,
+                          "tflops": tf, "pct_of_spec_bf16_peak": 100 * tf / SPEC_BF16_TFLOPS,
+                          "data": "torch.randn bf16 (timing only)"}), flush=True)
+        del q, k, v, o, lse
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} at {where}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -395,7 +440,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["all", "main"], default="all",
                     help="main: time only the bf16 non-causal step (for profiler runs)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print TFLOP/s for the sequence sweep and the long-context case instead")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
