@@ -66,7 +66,10 @@ typedef enum {
  *   q, k, v : [B][H][N][d] bf16 or fp16 (per `dtype`), read only.
  *   o       : [B][H][N][d] same dtype, written.
  *   lse     : [B][H][N] fp32, written; may be NULL (then not written).
- *   B, H, N : >= 1, B*H*N < 2^31.   d : 64, 128 or 256.
+ *   B, H, N : >= 1, B*H*N < 2^31.
+ *   d       : a multiple of 8, at most 256.  64, 128 and 256 run natively;
+ *             other sizes run zero-padded to the next of those (the padding
+ *             adds zero terms to every score and is never stored).
  *   scale   : finite and > 0 (usually 1/sqrt(d)).
  *   causal  : 0 or 1 (key j visible to query i iff j <= i).
  * Rounding: scores, statistics and accumulation are fp32; P is rounded to

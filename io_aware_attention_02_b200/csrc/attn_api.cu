@@ -209,7 +209,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   attn_status_t r = common_checks(B, H, N, scale, causal);
   if (r != ATTN_OK) return r;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  // any multiple of 8 up to 256 (16-byte rows for TMA); run as 64, 128 or 256
+  if (d > 256 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);
   if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
@@ -225,9 +227,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if ((r = make_map(&p.tm_k, k, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
   if ((r = make_map(&p.tm_v, v, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
   fill_common(&p, st, lse, o, BH, N, scale);
+  p.d_out = d;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 256) {
+  if (dk == 256) {
     if (dtype == ATTN_BF16)
       return causal ? launch_fwd256<__nv_bfloat16, true>(p, st->sm_count, s)
                     : launch_fwd256<__nv_bfloat16, false>(p, st->sm_count, s);
@@ -235,10 +238,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                   : launch_fwd256<__half, false>(p, st->sm_count, s);
   }
   if (dtype == ATTN_BF16)
-    return d == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
-                   : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
-  return d == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
-                 : launch_fwd_c<__half, 128>(p, grid, causal, s);
+    return dk == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
+                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
+  return dk == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
+                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
 }
 
 attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int H, int N, int d,
@@ -294,6 +297,7 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   p.k_desc = k_descale;
   p.v_desc = v_descale;
   fill_common(&p, st, lse, o, BH, N, scale);
+  p.d_out = d;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (v_transpose)
@@ -379,6 +383,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = wait_limit_ns();
   p.fault = 0;
+  p.d_out = d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the record keeps the previous call's contents: it must start at zero
   if (cudaMemsetAsync(st->scratch, 0, kNoAllocStatusBytes, s) != cudaSuccess) return ATTN_ERR_CUDA;

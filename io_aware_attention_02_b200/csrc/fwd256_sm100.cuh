@@ -337,7 +337,9 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.N + row) * D;
+      // O rows are d_out wide (d_out <= D: smaller head dims run zero-padded
+      // to D; the padding columns of O are zero and are not stored)
+      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.N + row) * p.d_out;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];
@@ -349,9 +351,10 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
           pk[i] = pack2<T>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
         if (row < p.N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+          const int groups = min(4, (p.d_out - cc * 32) >> 3);   // 8 values per 16-byte store
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            if (i < groups) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
       if (p.lse != nullptr && row < p.N)

@@ -66,7 +66,8 @@ def _fwd(lib, q=GOOD, k=GOOD, v=GOOD, o=GOOD, lse=None, B=1, H=1, N=128, d=64, s
     (dict(scale=float("inf")), binding.ATTN_ERR_INVALID_ARG),
     (dict(causal=2), binding.ATTN_ERR_INVALID_ARG),
     (dict(d=0), binding.ATTN_ERR_INVALID_ARG),
-    (dict(d=96), binding.ATTN_ERR_UNSUPPORTED),
+    (dict(d=100), binding.ATTN_ERR_UNSUPPORTED),
+    (dict(d=264), binding.ATTN_ERR_UNSUPPORTED),
     (dict(d=512), binding.ATTN_ERR_UNSUPPORTED),
     (dict(dtype=7), binding.ATTN_ERR_UNSUPPORTED),
     (dict(q=GOOD + 8), binding.ATTN_ERR_MISALIGNED),

@@ -30,6 +30,25 @@ def test_ragged_and_multi_tile(lib, d, causal, N):
     assert_bf16_ok(err, (N, d, causal))
 
 
+@pytest.mark.parametrize("d", [8, 40, 96, 136, 200, 248])
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dims_padded(lib, d, causal):
+    """Head dims that are not 64, 128 or 256 run zero-padded to the next of
+    those (the padding changes no score and no stored column)."""
+    err, _ = run_and_compare(lib, 1, 3, 333, d, causal, seed=d)
+    assert_bf16_ok(err, ("d", d, causal))
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_hidden_2048_sweep_shape(lib, d):
+    """Sweep shapes with hidden size 2048 (H = 2048 / d), total tokens 16K."""
+    N = 2048
+    rows = inputs.sample_rows(N, 32, seed=7)
+    err, _ = run_and_compare(lib, 16384 // N, 2048 // d, N, d, True, rows=rows,
+                             heads=[(0, 0), (7, 2048 // d - 1)])
+    assert_bf16_ok(err, ("hidden 2048", d))
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_fp16(lib, d, causal):
