@@ -121,3 +121,32 @@ def test_v_transpose_matches_mn_major(lib, causal, N):
     assert torch.equal(o0, o1) and torch.equal(l0, l1)
     o_ref, _ = A.attention(q, k, v, 1 / math.sqrt(128), causal)
     assert errors(o1.cpu(), None, o_ref, None)["rmse"] <= FP8_RMSE
+
+
+def test_accuracy_vs_low_precision_baselines(lib):
+    """The pages' accuracy experiment (outlier inputs): FP8 with per-block
+    scales and Hadamard rotation is more accurate than a per-tensor FP8
+    attention, and the fp16 kernel (fp32 statistics) more accurate than a
+    standard fp16 attention that writes its softmax out in fp16.  The pages
+    report 2.6x and 1.7x; here only the direction is asserted."""
+    from oracle import baselines as Bl
+    N, d = 1024, 128
+    scale = 1 / math.sqrt(d)
+    q, k, v = _x(1, 2, N, d, seed=77)
+    signs = torch.from_numpy(inputs.hadamard_signs(d, seed=5))
+    o8, _, _ = _fp8_attention(lib, q, k, v, False, True, inputs.hadamard_signs(d, seed=5))
+    q16, k16, v16 = (t.to(torch.float16) for t in (q, k, v))
+    o16, _ = lib.fwd(q16.cuda(), k16.cuda(), v16.cuda(), scale=scale)
+    torch.cuda.synchronize()
+    e8, e8b, e16, e16b = [], [], [], []
+    for h in range(2):
+        qq, kk, vv = (t[0, h].double().numpy() for t in (q, k, v))
+        o_ref, _ = A.attention_head(qq, kk, vv, scale)
+        e8.append(Bl.rmse(o8[0, h].double().cpu().numpy(), o_ref))
+        e8b.append(Bl.rmse(Bl.per_tensor_fp8_attention(qq, kk, vv, scale), o_ref))
+        q6, k6, v6 = (t[0, h].double().numpy() for t in (q16, k16, v16))
+        o_ref16, _ = A.attention_head(q6, k6, v6, scale)
+        e16.append(Bl.rmse(o16[0, h].double().cpu().numpy(), o_ref16))
+        e16b.append(Bl.rmse(Bl.standard_fp16_attention(q6, k6, v6, scale), o_ref16))
+    assert np.mean(e8) < np.mean(e8b), (e8, e8b)
+    assert np.mean(e16) < np.mean(e16b), (e16, e16b)

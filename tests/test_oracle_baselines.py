@@ -1,0 +1,54 @@
+"""Pins for the low-precision baselines of the pages' accuracy experiment
+(CPU only)."""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention as A
+from oracle import baselines as Bl
+from oracle import fp8 as F
+from io_aware_attention_02_b200 import inputs
+
+
+def test_baselines_exact_on_representable_uniform_case():
+    """Q = 0 gives uniform attention; with N = 4 and V rows 0, 1, 2, 4 every
+    rounding step lands on a representable value (V / (4/448) = 0, 112, 224,
+    448 in e4m3; P = 1/4), so both baselines return the exact output."""
+    q = np.zeros((4, 8))
+    k = np.random.default_rng(0).standard_normal((4, 8))
+    v = np.tile(np.array([0.0, 1.0, 2.0, 4.0])[:, None], (1, 8))
+    o_ref, _ = A.attention_head(q, k, v, 0.5)
+    np.testing.assert_array_equal(Bl.standard_fp16_attention(q, k, v, 0.5), o_ref)
+    np.testing.assert_array_equal(Bl.per_tensor_fp8_attention(q, k, v, 0.5), o_ref)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_baselines_close_but_not_exact_on_gaussian(causal):
+    x = [inputs.head_f32(0, t, 0, 0, 256, 64).astype(np.float64) for t in "qkv"]
+    o_ref, _ = A.attention_head(*x, 1 / 8, causal)
+    e16 = Bl.rmse(Bl.standard_fp16_attention(*x, 1 / 8, causal), o_ref)
+    e8 = Bl.rmse(Bl.per_tensor_fp8_attention(*x, 1 / 8, causal), o_ref)
+    assert 0 < e16 < 2e-3
+    assert e16 < e8 < 0.1
+
+
+def test_block_quantisation_with_rotation_beats_per_tensor_on_outliers():
+    """The mechanism behind the pages' FP8 claim, on the CPU: quantising Q,
+    K, V per 128-row block (Q and K rotated first) loses less than one scale
+    per tensor when 0.1 % of the entries are large outliers."""
+    N, d = 512, 128
+    x = [inputs.head_f32(1, t, 0, 0, N, d, outliers=True).astype(np.float64) for t in "qkv"]
+    scale = 1 / math.sqrt(d)
+    o_ref, _ = A.attention_head(*x, scale)
+    e_tensor = Bl.rmse(Bl.per_tensor_fp8_attention(*x, scale), o_ref)
+    signs = inputs.hadamard_signs(d, seed=0)
+    deq = []
+    for t, xx in zip("qkv", x):
+        rot = t != "v"
+        c, s, _ = F.quantize_blocks(xx[None, None], rot, signs)
+        deq.append(F.dequantize_blocks(c, s)[0, 0])
+    o_blk, _ = A.attention_head(*deq, scale)
+    e_block = Bl.rmse(o_blk, o_ref)
+    assert e_block < e_tensor / 1.5, (e_block, e_tensor)
