@@ -101,6 +101,13 @@ attn_status_t common_checks(int B, int H, int N, float scale, int causal) {
   return ATTN_OK;
 }
 
+// Work distribution (see sched_unit / decode_unit in fwd_sm100.cuh):
+// `n_blocks` row blocks per head, `grid` persistent CTAs.
+void set_schedule(attn::FwdParams* p, int causal, int n_blocks, int grid) {
+  p->snake = causal ? 1 : 0;
+  p->order = (causal && n_blocks < grid) ? 1 : 0;
+}
+
 template <typename E, int D, bool CAUSAL, bool VT = false>
 attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<E, D>;
@@ -137,6 +144,7 @@ attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream
   p.n_qpairs = (p.N + 127) / 128;
   p.n_units = p.BH * p.n_qpairs;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
+  set_schedule(&p, CAUSAL ? 1 : 0, p.n_qpairs, grid);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -229,6 +237,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   fill_common(&p, st, lse, o, BH, N, scale);
   p.d_out = d;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  set_schedule(&p, causal, p.n_qpairs, grid);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dk == 256) {
     if (dtype == ATTN_BF16)
@@ -299,6 +308,7 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   fill_common(&p, st, lse, o, BH, N, scale);
   p.d_out = d;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  set_schedule(&p, causal, p.n_qpairs, grid);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (v_transpose)
     return causal ? launch_fwd<__nv_fp8_e4m3, 128, true, true>(p, grid, s)
@@ -388,6 +398,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   // the record keeps the previous call's contents: it must start at zero
   if (cudaMemsetAsync(st->scratch, 0, kNoAllocStatusBytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  set_schedule(&p, causal, p.n_qpairs, grid);
   if (dtype == ATTN_BF16)
     return d == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);

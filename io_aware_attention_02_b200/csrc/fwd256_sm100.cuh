@@ -110,10 +110,11 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       uint32_t kv_iter = 0, unit_iter = 0;
       int64_t skipped = -1;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
-        const int bh = unit / n_qt;
-        const int qr = unit % n_qt;
-        const int qt = CAUSAL ? (n_qt - 1 - qr) : qr;
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh, qt;
+        decode_unit<CAUSAL>(unit, n_qt, p.BH, p.order, bh, qt);
         const int n = CAUSAL ? min(qt + 1, n_kv) : n_kv;
         ok = mbar_wait(q_empty, (unit_iter & 1) ^ 1, p.status, abort_flag, kWhereQEmpty, lim);
         if (!ok) break;
@@ -187,9 +188,12 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         return r;
       };
 
-      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
-        const int qr = unit % n_qt;
-        const int qt = CAUSAL ? (n_qt - 1 - qr) : qr;
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh_, qt;
+        decode_unit<CAUSAL>(unit, n_qt, p.BH, p.order, bh_, qt);
+        (void)bh_;
         const int n = CAUSAL ? min(qt + 1, n_kv) : n_kv;
         const uint32_t base = kv_iter;  // K_j at base + seq_k(j), V_j at base + seq_v(j, n)
         ok = mbar_wait(q_full, unit_iter & 1, p.status, abort_flag, kWhereQFull, lim);
@@ -239,10 +243,11 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
     bool ok = true;
     constexpr float kLazy = 8.0f;
 
-    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
-      const int bh = unit / n_qt;
-      const int qr = unit % n_qt;
-      const int qt = CAUSAL ? (n_qt - 1 - qr) : qr;
+    for (int k = 0; ok; ++k) {
+      const int unit = sched_unit(k, p.snake);
+      if (unit >= p.n_units) break;
+      int bh, qt;
+      decode_unit<CAUSAL>(unit, n_qt, p.BH, p.order, bh, qt);
       const int n = CAUSAL ? min(qt + 1, n_kv) : n_kv;
       const int row = qt * 128 + row_in_tile;
       const float c = p.scale_log2;

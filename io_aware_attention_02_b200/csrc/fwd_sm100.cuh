@@ -13,7 +13,8 @@
 //
 // Structure (Blackwell-native; the pages' Hopper WGMMA design is prior art):
 //   * persistent grid, one CTA per SM, work unit = (batch*head, 256 query rows)
-//     = two 128-row Q tiles ("slots");
+//     = two 128-row Q tiles ("slots"); causal units are taken longest first
+//     and dealt to the CTAs in a snake order for balance;
 //   * warp 0: TMA producer -- Q tiles once per unit, then K_j, V_j through a
 //     multi-stage shared-memory ring guarded by full/empty mbarriers
 //     (producer/consumer warp specialisation: dibro.site, "Arquitectura y
@@ -88,6 +89,8 @@ struct FwdParams {
   int* status;       // 4-int device status word
   int BH, N, n_kv, n_qpairs, n_units;
   int d_out;         // head dim of the tensors (<= the kernel's D; columns beyond it read as zero)
+  int snake;         // work distribution: alternate round direction (causal)
+  int order;         // 1 = longest-first across heads (causal, short heads)
   float scale_log2;  // scale * log2(e)
   unsigned long long wait_limit_ns;
   int fault;         // test hook: 1 = CTA 0 skips its first K load (waits must run out)
@@ -116,6 +119,34 @@ struct FwdCfg {
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + 1 KiB alignment slack
 };
+
+// Work distribution.  The persistent CTAs walk the unit list in rounds of
+// gridDim.x units.  Non-causal units all cost the same: plain rounds, in
+// head-major order, so the CTAs of a round share one head's K/V in L2.
+// Causal units get longer with the row block: the rounds alternate direction
+// (a snake), which over a longest-first list gives every CTA a near-equal
+// share.  Longest first is taken across heads when a head has fewer units
+// than there are CTAs, and within each head otherwise (then every running
+// CTA streams the same head's K/V).
+__device__ __forceinline__ int sched_unit(int k, int snake) {
+  const int r = (snake && (k & 1)) ? static_cast<int>(gridDim.x - 1 - blockIdx.x)
+                                   : static_cast<int>(blockIdx.x);
+  return k * static_cast<int>(gridDim.x) + r;
+}
+
+// unit -> (batch*head, block of query rows); order 1 = longest first across
+// heads (causal only).
+template <bool CAUSAL>
+__device__ __forceinline__ void decode_unit(int unit, int n_blocks, int BH, int order, int& bh, int& blk) {
+  if (CAUSAL && order == 1) {
+    blk = n_blocks - 1 - unit / BH;
+    bh = unit % BH;
+  } else {
+    bh = unit / n_blocks;
+    blk = unit % n_blocks;
+    if (CAUSAL) blk = n_blocks - 1 - blk;
+  }
+}
 
 // Barrier ids reported on timeout (status[1]).
 enum : int {
@@ -348,10 +379,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       uint32_t kv_iter = 0, unit_iter = 0;
       int64_t skipped = -1;
       bool ok = true;
-      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
-        const int bh = unit / p.n_qpairs;
-        const int qr = unit % p.n_qpairs;
-        const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh, qp;
+        decode_unit<CAUSAL>(unit, p.n_qpairs, p.BH, p.order, bh, qp);
         const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
         ok = mbar_wait(q_empty, (unit_iter & 1) ^ 1, p.status, abort_flag, kWhereQEmpty, lim);
         if (!ok) break;
@@ -474,9 +506,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         }
       };
 
-      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++unit_iter) {
-        const int qr = unit % p.n_qpairs;
-        const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh_, qp;
+        decode_unit<CAUSAL>(unit, p.n_qpairs, p.BH, p.order, bh_, qp);
+        (void)bh_;
         const int n0 = CAUSAL ? min(2 * qp + 1, n_kv) : n_kv;
         const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
         const uint32_t base = kv_iter;  // K_j at base + 2j, V_j at base + 2j + 1
@@ -540,9 +575,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
     const int tt = threadIdx.x - 64;              // 0..63
     uint32_t kv_iter = 0, v_cnt = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
-      const int qr = unit % p.n_qpairs;
-      const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+    for (int k = 0; ok; ++k) {
+      const int unit = sched_unit(k, p.snake);
+      if (unit >= p.n_units) break;
+      int bh_, qp;
+      decode_unit<CAUSAL>(unit, p.n_qpairs, p.BH, p.order, bh_, qp);
+      (void)bh_;
       const int n1 = CAUSAL ? min(2 * qp + 2, n_kv) : n_kv;
       for (int j = 0; j < n1; ++j, ++v_cnt) {
         const uint32_t iv = kv_iter + 2 * j + 1;
@@ -581,10 +619,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
     constexpr float kPGain = 256.0f;
     constexpr float kLazy = kF8 ? 0.75f : 8.0f;
 
-    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
-      const int bh = unit / p.n_qpairs;
-      const int qr = unit % p.n_qpairs;
-      const int qp = CAUSAL ? (p.n_qpairs - 1 - qr) : qr;
+    for (int k = 0; ok; ++k) {
+      const int unit = sched_unit(k, p.snake);
+      if (unit >= p.n_units) break;
+      int bh, qp;
+      decode_unit<CAUSAL>(unit, p.n_qpairs, p.BH, p.order, bh, qp);
       const int nt = CAUSAL ? min(2 * qp + t + 1, n_kv) : n_kv;
       const int row = qp * 256 + t * 128 + row_in_tile;
       float m = -INFINITY, l = 0.f;
