@@ -80,6 +80,24 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        void* stream);
 
 /*
+ * attn_fwd_strided -- attn_fwd over strided views.  The pages' kernel
+ * signature takes (batch, head, sequence) strides for Q, K, V and the output
+ * ("FlashAttention-3 warp specialization on Hopper", vikram-blog.pages.dev,
+ * "Production Implementation & Code Pattern"); this entry point does the
+ * same, so e.g. [B][N][H][d] (BSHD) tensors need no copy.
+ *   x_strides : 3 element strides of tensor x over (batch, head, row), host
+ *               array; the head dim is contiguous.  Each stride must be a
+ *               positive multiple of 8 elements (16 bytes) and the row
+ *               stride at least d.  O's rows must not overlap one another.
+ *   Everything else as attn_fwd (lse stays contiguous [B][H][N]).
+ */
+attn_status_t attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int N, int d, const long long* q_strides,
+                               const long long* k_strides, const long long* v_strides,
+                               const long long* o_strides, float scale, int causal, int dtype,
+                               void* stream);
+
+/*
  * attn_quant_fp8 -- per-block e4m3 quantisation with optional incoherent
  * processing (quantum-bit repost "H100 utilisation 75% ... FlashAttention-3",
  * third technical upgrade: block-wise quantisation and incoherent processing;

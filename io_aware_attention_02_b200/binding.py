@@ -30,6 +30,7 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_debug_set_fault": (_I, [_I, _I]),
     "attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_fwd_strided": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _F, _I, _I, _P]),
 }
 
 
@@ -91,26 +92,50 @@ def _check_qkv(q, k, v):
         raise ValueError("q, k, v must have the same shape")
 
 
+def _strides3(t):
+    """(batch, head, row) element strides of a [B, H, N, d] view with a
+    contiguous head dim, as a ctypes array."""
+    if t.stride(-1) != 1:
+        raise ValueError("the head dim (last) must be contiguous")
+    return (ctypes.c_longlong * 3)(*t.stride()[:3])
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: float | None = None, out: torch.Tensor | None = None,
         lse: torch.Tensor | None = None, return_lse: bool = True):
-    """O, LSE = attention(q, k, v) through ``attn_fwd`` on the current stream.
+    """O, LSE = attention(q, k, v) on the current stream.
 
-    q, k, v: contiguous CUDA tensors [B, H, N, d] of bf16 or fp16.
+    q, k, v: CUDA tensors [B, H, N, d] of bf16 or fp16.  Contiguous tensors go
+    through ``attn_fwd``; other views with a contiguous head dim (for example
+    ``x.transpose(1, 2)`` of a [B, N, H, d] tensor) through
+    ``attn_fwd_strided``, without a copy.  ``out`` may be such a view too.
     Returns (o, lse) with lse fp32 [B, H, N] (None if ``return_lse`` is False).
     """
-    _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D [B, H, N, d]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
     if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must all be bf16 or all fp16")
     B, H, N, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    o = torch.empty_like(q) if out is None else out
+    o = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
-    code = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse) if return_lse else None,
-                           B, H, N, d, scale, int(bool(causal)), dtype, _stream(q.device))
-    _check("attn_fwd", code)
+    lse_p = _ptr(lse) if return_lse else None
+    if all(t.is_contiguous() for t in (q, k, v, o)):
+        code = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), lse_p, B, H, N, d, scale,
+                               int(bool(causal)), dtype, _stream(q.device))
+        _check("attn_fwd", code)
+    else:
+        code = load().attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), lse_p, B, H, N, d,
+                                       _strides3(q), _strides3(k), _strides3(v), _strides3(o),
+                                       scale, int(bool(causal)), dtype, _stream(q.device))
+        _check("attn_fwd_strided", code)
     return o, (lse if return_lse else None)
 
 

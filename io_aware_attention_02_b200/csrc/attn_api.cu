@@ -65,19 +65,37 @@ attn_status_t device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 3-D tiled map over a contiguous [BH][N][D] tensor: box = (box_cols, 128, 1),
-// 128-byte swizzle; out-of-range rows read as zero.
+// Element strides of a [B][H][N][d] view over (batch, head, row); the head
+// dim is contiguous.
+struct Strides {
+  long long b, h, n;
+};
+Strides contiguous(int H, int N, int d) {
+  return {static_cast<long long>(H) * N * d, static_cast<long long>(N) * d, d};
+}
+
+// Strides TMA can use: positive multiples of 16 bytes, rows not overlapping
+// (n >= d).
+bool strides_ok(const Strides& s, int d, int esize) {
+  const long long a[3] = {s.b, s.h, s.n};
+  for (long long x : a)
+    if (x <= 0 || (x * esize) % 16 != 0) return false;
+  return s.n >= d;
+}
+
+// 4-D tiled map over (d, N, H, B) with the given strides: box = (box_cols,
+// 128, 1, 1), 128-byte swizzle; out-of-range rows and columns read as zero.
 attn_status_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize,
-                       int BH, int N, int D, int box_cols) {
+                       int B, int H, int N, int D, const Strides& st, int box_cols) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return ATTN_ERR_CUDA;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esize,
-                           static_cast<cuuint64_t>(N) * D * esize};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), 128u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.n) * esize, static_cast<cuuint64_t>(st.h) * esize,
+                           static_cast<cuuint64_t>(st.b) * esize};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), 128u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
@@ -150,13 +168,15 @@ attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream
 }
 
 // Fills the fields shared by the 16-bit and FP8 launches.
-attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void* o, int BH, int N,
-                          float scale) {
+attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void* o, int BH, int H,
+                          int N, float scale) {
   p->o = o;
   p->lse = lse;
   p->status = st->status;
   p->BH = BH;
   p->N = N;
+  p->H = H;
+  p->o_sb = p->o_sh = p->o_sn = 0;   // O strides: set by each caller
   p->n_kv = (N + 127) / 128;
   p->n_qpairs = (N + 255) / 256;
   p->n_units = BH * p->n_qpairs;
@@ -169,6 +189,55 @@ attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void*
   g_fault_mode = 0;
   g_fault_limit_ms = 0;
   return ATTN_OK;
+}
+
+// 16-bit forward over strided [B][H][N][d] views (head dim contiguous).
+attn_status_t fwd16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, const Strides& sq, const Strides& sk, const Strides& sv,
+                    const Strides& so, float scale, int causal, int dtype, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  // any multiple of 8 up to 256 (16-byte rows for TMA); run as 64, 128 or 256
+  if (d > 256 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (!strides_ok(sq, d, 2) || !strides_ok(sk, d, 2) || !strides_ok(sv, d, 2) || !strides_ok(so, d, 2))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+
+  DeviceState* st = nullptr;
+  if ((r = device_state(&st)) != ATTN_OK) return r;
+
+  const int BH = B * H;
+  const CUtensorMapDataType dt =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  attn::FwdParams p{};
+  if ((r = make_map(&p.tm_q, q, dt, 2, B, H, N, d, sq, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, B, H, N, d, sk, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, B, H, N, d, sv, 64)) != ATTN_OK) return r;
+  fill_common(&p, st, lse, o, BH, H, N, scale);
+  p.d_out = d;
+  p.o_sb = so.b;
+  p.o_sh = so.h;
+  p.o_sn = so.n;
+  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  set_schedule(&p, causal, p.n_qpairs, grid);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dk == 256) {
+    if (dtype == ATTN_BF16)
+      return causal ? launch_fwd256<__nv_bfloat16, true>(p, st->sm_count, s)
+                    : launch_fwd256<__nv_bfloat16, false>(p, st->sm_count, s);
+    return causal ? launch_fwd256<__half, true>(p, st->sm_count, s)
+                  : launch_fwd256<__half, false>(p, st->sm_count, s);
+  }
+  if (dtype == ATTN_BF16)
+    return dk == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
+                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
+  return dk == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
+                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
 }
 
 }  // namespace
@@ -213,44 +282,22 @@ attn_status_t attn_last_status(void* stream, int* where) {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, float scale, int causal, int dtype, void* stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
-  attn_status_t r = common_checks(B, H, N, scale, causal);
-  if (r != ATTN_OK) return r;
-  if (d < 1) return ATTN_ERR_INVALID_ARG;
-  // any multiple of 8 up to 256 (16-byte rows for TMA); run as 64, 128 or 256
-  if (d > 256 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
-  const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);
-  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
-  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  const Strides c = contiguous(H, N, d);
+  return fwd16(q, k, v, o, lse, B, H, N, d, c, c, c, c, scale, causal, dtype, stream);
+}
 
-  DeviceState* st = nullptr;
-  if ((r = device_state(&st)) != ATTN_OK) return r;
-
-  const int BH = B * H;
-  const CUtensorMapDataType dt =
-      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  attn::FwdParams p{};
-  if ((r = make_map(&p.tm_q, q, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_k, k, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_v, v, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
-  fill_common(&p, st, lse, o, BH, N, scale);
-  p.d_out = d;
-  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
-  set_schedule(&p, causal, p.n_qpairs, grid);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dk == 256) {
-    if (dtype == ATTN_BF16)
-      return causal ? launch_fwd256<__nv_bfloat16, true>(p, st->sm_count, s)
-                    : launch_fwd256<__nv_bfloat16, false>(p, st->sm_count, s);
-    return causal ? launch_fwd256<__half, true>(p, st->sm_count, s)
-                  : launch_fwd256<__half, false>(p, st->sm_count, s);
-  }
-  if (dtype == ATTN_BF16)
-    return dk == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
-                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
-  return dk == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
-                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
+attn_status_t attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int N, int d, const long long* q_strides,
+                               const long long* k_strides, const long long* v_strides,
+                               const long long* o_strides, float scale, int causal, int dtype,
+                               void* stream) {
+  if (q_strides == nullptr || k_strides == nullptr || v_strides == nullptr || o_strides == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  const Strides sq{q_strides[0], q_strides[1], q_strides[2]};
+  const Strides sk{k_strides[0], k_strides[1], k_strides[2]};
+  const Strides sv{v_strides[0], v_strides[1], v_strides[2]};
+  const Strides so{o_strides[0], o_strides[1], o_strides[2]};
+  return fwd16(q, k, v, o, lse, B, H, N, d, sq, sk, sv, so, scale, causal, dtype, stream);
 }
 
 attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int H, int N, int d,
@@ -299,14 +346,18 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   const int BH = B * H;
   attn::FwdParams p{};
   const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  if ((r = make_map(&p.tm_q, q8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_k, k8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_v, v8, dt, 1, BH, N, d, 128)) != ATTN_OK) return r;
+  const Strides c8 = contiguous(H, N, d);
+  if ((r = make_map(&p.tm_q, q8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
   p.q_desc = q_descale;
   p.k_desc = k_descale;
   p.v_desc = v_descale;
-  fill_common(&p, st, lse, o, BH, N, scale);
+  fill_common(&p, st, lse, o, BH, H, N, scale);
   p.d_out = d;
+  p.o_sb = c8.b;
+  p.o_sh = c8.h;
+  p.o_sn = c8.n;
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   set_schedule(&p, causal, p.n_qpairs, grid);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -379,14 +430,19 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   const CUtensorMapDataType dt =
       dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   attn::FwdParams p{};
-  if ((r = make_map(&p.tm_q, q, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_k, k, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_v, v, dt, 2, BH, N, d, 64)) != ATTN_OK) return r;
+  const Strides cs = contiguous(H, N, d);
+  if ((r = make_map(&p.tm_q, q, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
   p.o = o;
   p.lse = lse;
   p.status = st->scratch;
   p.BH = BH;
+  p.H = H;
   p.N = N;
+  p.o_sb = cs.b;
+  p.o_sh = cs.h;
+  p.o_sn = cs.n;
   p.n_kv = (N + 127) / 128;
   p.n_qpairs = (N + 255) / 256;
   p.n_units = BH * p.n_qpairs;

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_3d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * 64, qt * 128, bh);
+          tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * 64, qt * 128, bh % p.H, bh / p.H);
         for (int q = 0; q < 2 * n && ok; ++q, ++kv_iter) {
           // q -> (K or V, key tile j), inverse of seq_k / seq_v
           const bool is_v = (q == 2 * n - 1) || (q > 0 && (q & 1) == 0);
@@ -135,8 +135,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
           mbar_arrive_expect_tx(kv_full + s, Cfg::kTileBytes);
           const CUtensorMap* map = is_v ? &p.tm_v : &p.tm_k;
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_3d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
-                        c * 64, j * 128, bh);
+            tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
+                        c * 64, j * 128, bh % p.H, bh / p.H);
         }
       }
       if (!ok) {
@@ -343,8 +343,10 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       tc_fence_after();
       const float inv_l = 1.0f / l;
       // O rows are d_out wide (d_out <= D: smaller head dims run zero-padded
-      // to D; the padding columns of O are zero and are not stored)
-      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.N + row) * p.d_out;
+      // to D; the padding columns of O are zero and are not stored); O may be
+      // strided over (batch, head, row)
+      T* orow = reinterpret_cast<T*>(p.o) + static_cast<int64_t>(bh / p.H) * p.o_sb +
+                static_cast<int64_t>(bh % p.H) * p.o_sh + static_cast<int64_t>(row) * p.o_sn;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];

@@ -30,7 +30,7 @@ def lib():
 def test_header_declares_the_boundary():
     assert _declared() == sorted(["attn_fwd", "attn_quant_fp8", "attn_fwd_fp8", "attn_last_status",
                                   "attn_status_string", "attn_debug_set_fault",
-                                  "attn_fwd_noalloc"])
+                                  "attn_fwd_noalloc", "attn_fwd_strided"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -94,6 +94,17 @@ def test_quant_and_fp8_validation(lib):
     assert F(*bad) == binding.ATTN_ERR_MISALIGNED
     bad = list(args); bad[14] = 3
     assert F(*bad) == binding.ATTN_ERR_INVALID_ARG
+
+
+def test_strided_validation(lib):
+    F = lib.attn_fwd_strided
+    ok = (ctypes.c_longlong * 3)(16 * 128 * 64, 128 * 64, 64)
+    bad_align = (ctypes.c_longlong * 3)(16 * 128 * 64, 128 * 64, 68)
+    overlap = (ctypes.c_longlong * 3)(16 * 128 * 64, 128 * 64, 32)
+    args = lambda qs: [GOOD] * 4 + [None, 1, 16, 128, 64, qs, ok, ok, ok, 0.125, 0, 0, None]
+    assert F(*args(None)) == binding.ATTN_ERR_INVALID_ARG
+    assert F(*args(bad_align)) == binding.ATTN_ERR_INVALID_ARG
+    assert F(*args(overlap)) == binding.ATTN_ERR_INVALID_ARG
 
 
 def test_debug_hook_validation(lib):

@@ -185,3 +185,39 @@ def test_lse_may_be_omitted_and_stream_respected(lib):
     torch.cuda.synchronize()
     assert torch.equal(o, o2)
     assert lib.last_status()[0] == 0
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True), (256, False), (96, True)])
+def test_strided_bshd_views_match_contiguous(lib, d, causal):
+    """[B, N, H, d] (BSHD) tensors passed as transposed views, and an output
+    written into a BSHD buffer, give bit-identical results to the contiguous
+    path; both match the oracle."""
+    B, H, N = 2, 3, 300
+    q, k, v = inputs.qkv(B, H, N, d, seed=21)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o_ref, l_ref = lib.fwd(qd, kd, vd, causal=causal)
+    qs, ks, vs = (t.transpose(1, 2).contiguous().transpose(1, 2) for t in (qd, kd, vd))
+    assert not qs.is_contiguous()
+    o_buf = torch.empty(B, N, H, d, dtype=q.dtype, device="cuda")
+    o_s, l_s = lib.fwd(qs, ks, vs, causal=causal, out=o_buf.transpose(1, 2))
+    torch.cuda.synchronize()
+    assert torch.equal(o_s, o_ref) and torch.equal(l_s, l_ref)
+    assert torch.equal(o_buf.transpose(1, 2), o_ref)
+    err = errors(o_s.cpu(), l_s.cpu(), *A.attention(q, k, v, 1 / math.sqrt(d), causal))
+    assert_bf16_ok(err, ("bshd", d))
+
+
+def test_strided_padded_rows_and_mixed_layouts(lib):
+    """Rows with padding between them (row stride > d) and a different layout
+    per tensor."""
+    B, H, N, d = 1, 2, 257, 64
+    q, k, v = inputs.qkv(B, H, N, d, seed=22)
+    big = torch.zeros(B, H, N, d + 32, dtype=q.dtype)
+    big[..., :d] = k
+    kp = big.cuda()[..., :d]                       # row stride d + 32
+    assert kp.stride(2) == d + 32
+    qs = q.transpose(1, 2).contiguous().cuda().transpose(1, 2)
+    o, lse = lib.fwd(qs, kp, v.cuda())
+    torch.cuda.synchronize()
+    err = errors(o.cpu(), lse.cpu(), *A.attention(q, k, v, 1 / math.sqrt(d), False))
+    assert_bf16_ok(err, "padded rows")
