@@ -29,6 +29,10 @@ Modules:
 * ``attention`` -- exact attention (the definition), probabilities, LSE.
 * ``fp8``       -- e4m3 rounding from the format's definition, Sylvester
   Hadamard matrix, per-block quantisation as the pages describe it.
+* ``backward``  -- gradients (dQ, dK, dV) of exact attention, the chain rule
+  written out.
+* ``baselines`` -- the per-tensor FP8 and standard FP16 attentions of the
+  pages' accuracy experiment.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 against closed forms, invariants, a hand-computed two-token example, a
@@ -37,4 +41,4 @@ pure-Python brute force and library routines (``torch`` SDPA in float64,
 print (2.6x, 1.7x) are NOT pinned: "parity unpinned" for those ratios.
 """
 
-from . import attention, fp8  # noqa: F401
+from . import attention, backward, baselines, fp8  # noqa: F401
