@@ -161,19 +161,6 @@ enum : int {
 
 // max of 128 values with 3-input max instructions, four independent chains.
 __device__ __forceinline__ float row_max128(const float (&s)[128]) {
-#if ATTN_MAX8
-  float a[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmax3(s[k], s[8 + k], s[16 + k]);
-#pragma unroll
-  for (int i = 24; i < 120; i += 16) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 8 + k]);
-  }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
-  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-#else
   float a[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
   for (int i = 4; i < 128; i += 8) {
@@ -181,7 +168,6 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
     for (int k = 0; k < 4; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 4 + k]);
   }
   return fmax3(fmaxf(a[0], a[1]), a[2], a[3]);
-#endif
 }
 
 // 2^x for a pair on the FMA pipe (Cody-Waite style split, then a minimax
@@ -219,13 +205,6 @@ __device__ __forceinline__ float2 exp2_mufu2(float2 x) {
   return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
-#ifndef ATTN_MAX8
-#define ATTN_MAX8 0
-#endif
-#ifndef ATTN_PUBDEFER
-#define ATTN_PUBDEFER 0
-#endif
-
 // Pairs i with (i % 8) < kPolyPairsPer8 take the polynomial path.
 constexpr int kPolyPairsPer8 = 1;
 
@@ -233,29 +212,6 @@ constexpr int kPolyPairsPer8 = 1;
 // packed to 16-bit pairs (or e4m3 quads, after the gain) and written over the
 // row's S columns in TMEM (32 columns per half at 16 bit, 16 at e4m3).
 // Returns the fp32 sum of the unrounded P of that half.
-// 16-bit half with a callback after the first kHookAt pairs (used to publish
-// the previous half once its TMEM store has had time to complete).
-template <typename T, bool kPoly, int kHookAt, typename Hook>
-__device__ __forceinline__ float exp_pack_half_hook(const float (&s)[128], int h, float c, float neg_m,
-                                                    uint32_t tS, Hook&& hook) {
-  const float2 c2 = make_float2(c, c);
-  const float2 nm2 = make_float2(neg_m, neg_m);
-  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  uint32_t pk[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    if (i == kHookAt) hook();
-    const int e = 64 * h + 2 * i;
-    const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, nm2);
-    const float2 pr = (kPoly && (i % 8) < kPolyPairsPer8) ? exp2_poly2<3>(x) : exp2_mufu2(x);
-    acc[i & 1] = __fadd2_rn(acc[i & 1], pr);
-    pk[i] = pack2<T>(pr.x, pr.y);
-  }
-  tmem_st32(tS + 32 * h, pk);
-  const float2 a = __fadd2_rn(acc[0], acc[1]);
-  return a.x + a.y;
-}
-
 template <bool kF8, typename T, bool kPoly>
 __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, float c, float neg_m,
                                                float pgain, uint32_t tS) {
@@ -746,30 +702,13 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         // to an exact 0; unmasked tiles may send part of their exp2 work to
         // the FMA pipe.
         float sum = 0.f;
-#if ATTN_PUBDEFER
-        if (!kF8 && !need_mask) {
-          // publish the first half once part of the second half has been
-          // issued, so the store of the first half completes under compute
-          sum = exp_pack_half<kF8, T, true>(s, 0, c, -m, pgain, tS);
-          sum += exp_pack_half_hook<T, true, ATTN_PUBDEFER>(s, 1, c, -m, tS, [&] {
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full + 2 * t + 0);
-          });
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          sum += need_mask ? exp_pack_half<kF8, T, false>(s, h, c, -m, pgain, tS)
+                           : exp_pack_half<kF8, T, true>(s, h, c, -m, pgain, tS);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(p_full + 2 * t + 1);
-        } else
-#endif
-        {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            sum += need_mask ? exp_pack_half<kF8, T, false>(s, h, c, -m, pgain, tS)
-                             : exp_pack_half<kF8, T, true>(s, h, c, -m, pgain, tS);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full + 2 * t + h);
-          }
+          mbar_arrive(p_full + 2 * t + h);
         }
         l = l * alpha + sum;
       }
