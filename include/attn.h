@@ -43,6 +43,8 @@
 #ifndef ATTN_SM100_H_
 #define ATTN_SM100_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -177,6 +179,50 @@ attn_status_t attn_last_status(void* stream, int* where);
 attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int N, int d, float scale, int causal, int dtype,
                                void* stream);
+
+/*
+ * attn_bwd_workspace_bytes -- size of the workspace attn_bwd needs:
+ * B * H * ceil(N / 128) * 256 * 4 bytes (two fp32 values per query row,
+ * rows padded to whole 128-row tiles).  Returns 0 for sizes < 1.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int N);
+
+/*
+ * attn_bwd -- 16-bit attention backward: the gradients of O with respect to
+ * Q, K and V, given dO.  The chain rule of the definition above, with the
+ * probabilities recomputed from the forward pass's LSE (P is never stored):
+ *
+ *   P  = exp(scale * Q K^T - LSE)   (0 where causal masking hides a key)
+ *   dV = P^T dO
+ *   dP = dO V^T,   D = rowsum(dO * O),   dS = P * (dP - D)
+ *   dQ = scale * dS K,   dK = scale * dS^T Q
+ *
+ * The pages benchmark this pass beside the forward (quantum-bit repost
+ * "H100 utilisation 75% ... FlashAttention-3", attention benchmark) without
+ * writing it out; these are the standard gradients of softmax attention.
+ *   q, k, v, o, d_o : [B][H][N][d] bf16 or fp16 (per `dtype`), read only;
+ *                     o and lse as returned by attn_fwd for the same q, k,
+ *                     v, scale and causal.
+ *   lse             : [B][H][N] fp32 (natural log), read only.
+ *   dq, dk, dv      : [B][H][N][d] same dtype, written.
+ *   workspace       : device memory of at least attn_bwd_workspace_bytes(B,
+ *                     H, N) bytes, 16-byte aligned, owned by the caller; its
+ *                     contents on entry do not matter and are overwritten
+ *                     (row statistics passed between the two kernels).
+ *   d               : a multiple of 8, at most 128 (64 and 128 natively,
+ *                     others zero-padded); larger d returns
+ *                     ATTN_ERR_UNSUPPORTED.
+ *   B, H, N, scale, causal, dtype, stream: as for attn_fwd.
+ * Rounding: scores, P, dP and accumulation are fp32; P and dS are rounded to
+ * the input dtype before the products that use them; D is accumulated in
+ * fp32 from the 16-bit dO and O; outputs are rounded to the input dtype.
+ * Deterministic (no atomics): two kernels on `stream`, the first writing
+ * dQ and the workspace, the second dK and dV.
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                       size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                       int dtype, void* stream);
 
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t s);

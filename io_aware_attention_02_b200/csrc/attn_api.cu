@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "bwd_sm100.cuh"
 #include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "quant_fp8.cuh"
@@ -240,6 +241,39 @@ attn_status_t fwd16(const void* q, const void* k, const void* v, void* o, float*
                   : launch_fwd_c<__half, 128>(p, grid, causal, s);
 }
 
+// Backward: the dQ kernel (which also writes the row statistics) then the
+// dK/dV kernel, on the same stream and the same persistent grid shape.
+template <typename E, int D, bool CAUSAL>
+attn_status_t launch_bwd(attn::BwdParams p, int sm_count, cudaStream_t stream) {
+  using Cfg = attn::BwdCfg<D>;
+  auto kq = attn::attn_bwd_dq_kernel<E, D, CAUSAL>;
+  auto kkv = attn::attn_bwd_dkdv_kernel<E, D, CAUSAL>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kDqSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kKvSmem) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_done = true;
+  }
+  p.n_units = p.BH * p.n_t;
+  const int grid = p.n_units < sm_count ? p.n_units : sm_count;
+  p.snake = CAUSAL ? 1 : 0;
+  p.order = (CAUSAL && p.n_t < grid) ? 1 : 0;
+  kq<<<grid, Cfg::kThreads, Cfg::kDqSmem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  kkv<<<grid, Cfg::kThreads, Cfg::kKvSmem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename E, int D>
+attn_status_t launch_bwd_c(const attn::BwdParams& p, int sm_count, int causal, cudaStream_t s) {
+  return causal ? launch_bwd<E, D, true>(p, sm_count, s) : launch_bwd<E, D, false>(p, sm_count, s);
+}
+
+size_t bwd_workspace_bytes(int B, int H, int N) {
+  return static_cast<size_t>(B) * H * ((N + 127) / 128) * 256 * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
@@ -460,4 +494,61 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
   return d == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
+}
+
+extern "C" size_t attn_bwd_workspace_bytes(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return bwd_workspace_bytes(B, H, N);
+}
+
+extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                  const void* d_o, const float* lse, void* dq, void* dk, void* dv,
+                                  void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                                  float scale, int causal, int dtype, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || d_o == nullptr || lse == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d > 128 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < bwd_workspace_bytes(B, H, N)) return ATTN_ERR_INVALID_ARG;
+  const void* p16[] = {q, k, v, o, d_o, dq, dk, dv, workspace};
+  for (const void* x : p16)
+    if (!aligned16(x)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+
+  DeviceState* st = nullptr;
+  if ((r = device_state(&st)) != ATTN_OK) return r;
+  const CUtensorMapDataType dt =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const Strides cs = contiguous(H, N, d);
+  attn::BwdParams p{};
+  if ((r = make_map(&p.tm_q, q, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_o, o, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_do, d_o, dt, 2, B, H, N, d, cs, 64)) != ATTN_OK) return r;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.lse = lse;
+  p.rows = static_cast<float*>(workspace);
+  p.status = st->status;
+  p.BH = B * H;
+  p.H = H;
+  p.N = N;
+  p.n_t = (N + 127) / 128;
+  p.d_out = d;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = wait_limit_ns();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int dk_ = d <= 64 ? 64 : 128;
+  if (dtype == ATTN_BF16)
+    return dk_ == 64 ? launch_bwd_c<__nv_bfloat16, 64>(p, st->sm_count, causal, s)
+                     : launch_bwd_c<__nv_bfloat16, 128>(p, st->sm_count, causal, s);
+  return dk_ == 64 ? launch_bwd_c<__half, 64>(p, st->sm_count, causal, s)
+                   : launch_bwd_c<__half, 128>(p, st->sm_count, causal, s);
 }

@@ -17,6 +17,8 @@ Recipe (the workloads of the FlashAttention-3 pages, synthetic):
   N(0, 10^2) term, which is the page's own wording.
 * The fp32 draws are rounded to bf16 (round-to-nearest-even, torch's CPU
   cast); that rounded tensor is what both the GPU and the oracle receive.
+* The output gradient dO of the backward pass is drawn the same way (tensor
+  id "do"), i.i.d. N(0, 1) rounded to the input dtype.
 * Hadamard sign diagonals (+-1 per head-dim entry) are drawn here too, so the
   random part of incoherent processing is an input to both sides.
 """
@@ -26,7 +28,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-_TENSOR_IDS = {"q": 0, "k": 1, "v": 2}
+_TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "do": 3}
 
 
 def _rng(seed: int, tensor: str, b: int, h: int) -> np.random.Generator:
@@ -74,6 +76,15 @@ def qkv(B: int, H: int, N: int, d: int, seed: int = 0, dtype=torch.bfloat16,
                 t[b, h] = torch.from_numpy(x).to(dtype)
         out.append(t)
     return tuple(out)
+
+
+def grad_out(B: int, H: int, N: int, d: int, seed: int = 0, dtype=torch.bfloat16) -> torch.Tensor:
+    """Output gradient dO, a CPU tensor [B, H, N, d] in ``dtype``."""
+    t = torch.empty((B, H, N, d), dtype=dtype)
+    for b in range(B):
+        for h in range(H):
+            t[b, h] = torch.from_numpy(head_f32(seed, "do", b, h, N, d)).to(dtype)
+    return t
 
 
 def sample_rows(N: int, count: int, seed: int = 0) -> np.ndarray:

@@ -30,7 +30,8 @@ def lib():
 def test_header_declares_the_boundary():
     assert _declared() == sorted(["attn_fwd", "attn_quant_fp8", "attn_fwd_fp8", "attn_last_status",
                                   "attn_status_string", "attn_debug_set_fault",
-                                  "attn_fwd_noalloc", "attn_fwd_strided"])
+                                  "attn_fwd_noalloc", "attn_fwd_strided", "attn_bwd",
+                                  "attn_bwd_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -105,6 +106,38 @@ def test_strided_validation(lib):
     assert F(*args(None)) == binding.ATTN_ERR_INVALID_ARG
     assert F(*args(bad_align)) == binding.ATTN_ERR_INVALID_ARG
     assert F(*args(overlap)) == binding.ATTN_ERR_INVALID_ARG
+
+
+def test_bwd_workspace_size(lib):
+    # two fp32 values per query row, rows padded to whole 128-row tiles
+    assert lib.attn_bwd_workspace_bytes(2, 3, 1) == 2 * 3 * 1 * 256 * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 129) == 2 * 256 * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 0) == 0
+
+
+def test_bwd_validation(lib):
+    F = lib.attn_bwd
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 256)
+
+    def call(**kw):
+        a = dict(q=GOOD, k=GOOD, v=GOOD, o=GOOD, do=GOOD, lse=GOOD, dq=GOOD, dk=GOOD, dv=GOOD,
+                 ws=GOOD, ws_bytes=ws, B=1, H=2, N=256, d=64, scale=0.125, causal=0, dtype=0)
+        a.update(kw)
+        return F(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"], a["ws"],
+                 a["ws_bytes"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["dtype"], None)
+
+    assert call(lse=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(ws=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(do=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(ws_bytes=ws - 4) == binding.ATTN_ERR_INVALID_ARG
+    assert call(N=0) == binding.ATTN_ERR_INVALID_ARG
+    assert call(causal=3) == binding.ATTN_ERR_INVALID_ARG
+    assert call(d=256) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(d=100) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(dtype=2) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(dk=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
+    assert call(ws=GOOD + 4) == binding.ATTN_ERR_MISALIGNED
+    assert call(lse=GOOD + 2) == binding.ATTN_ERR_MISALIGNED
 
 
 def test_debug_hook_validation(lib):

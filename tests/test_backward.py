@@ -1,0 +1,170 @@
+"""GPU parity of the backward kernels (attn_bwd) against the fp64 oracle's
+gradients, called through the C ABI on seeded synthetic inputs.
+
+Tolerance, from the kernel's rounding: P and dS are rounded to the input
+dtype before the products that use them and every output is rounded to it
+once, so each gradient carries about two bf16 roundings (unit roundoff
+2^-9, i.e. ~1.1e-3 RMS relative each).  A CPU emulation of exactly those
+roundings on these inputs gives an RMSE of 2.2e-3 to 2.5e-3 of the
+gradient's RMS and a maximum error of 2.4e-3 to 4.2e-3 of its largest
+entry (N 300 to 1000, d 64 and 128, causal and not).  The bounds below are
+four and five times that.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from io_aware_attention_02_b200 import inputs
+from oracle import backward as BK
+
+pytestmark = pytest.mark.gpu
+
+REL_RMSE = 1e-2        # RMSE / RMS(oracle)
+REL_MAX = 2e-2         # max |error| / max |oracle|
+# Gradients that vanish exactly (N = 1: dQ = dK = 0) are compared against
+# these floors instead: the natural size of a gradient entry here is 0.05-1.
+RMS_FLOOR = 1e-3
+MAX_FLOOR = 1e-2
+
+
+def _grad_errors(got, ref):
+    g = got.detach().to("cpu", torch.float64).numpy()
+    dif = g - ref
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return {"rel_rmse": float(np.sqrt(np.mean(dif ** 2))) / max(rms, RMS_FLOOR),
+            "rel_max": float(np.abs(dif).max()) / max(float(np.abs(ref).max()), MAX_FLOOR),
+            "finite": bool(np.isfinite(g).all())}
+
+
+def _assert_ok(err, what):
+    assert err["finite"], (what, err)
+    assert err["rel_rmse"] <= REL_RMSE, (what, err)
+    assert err["rel_max"] <= REL_MAX, (what, err)
+
+
+def _run(lib, B, H, N, d, causal, dtype=torch.bfloat16, seed=0, scale=None, heads=None):
+    q, k, v = inputs.qkv(B, H, N, d, seed=seed, dtype=dtype)
+    do = inputs.grad_out(B, H, N, d, seed=seed, dtype=dtype)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = lib.fwd(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = lib.bwd(qd, kd, vd, o, dod, lse, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    code, where = lib.last_status()
+    assert code == 0, where
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    out = []
+    for b, h in heads:
+        ref = BK.attention_backward_head(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq[b, h], dk[b, h], dv[b, h]), ref):
+            out.append(((b, h, name), _grad_errors(got, r)))
+    return out, (dq, dk, dv)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 100, 128, 129, 256, 257, 500])
+def test_ragged_and_multi_tile(lib, d, causal, N):
+    errs, _ = _run(lib, 1, 2, N, d, causal, seed=N)
+    for what, e in errs:
+        _assert_ok(e, (N, d, causal, what))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_token_closed_form(lib, causal):
+    """N = 1: P = 1, so dV = dO and dS = dO.v - dO.O = 0, hence dQ = dK = 0.
+
+    dV is exact (P = 1 is exact in 16 bits).  dQ and dK vanish up to the
+    difference of two fp32 sums of the same 128 products, dO.v by the tensor
+    cores and dO.O by the row threads (|dO.v| reaches ~40 here, and the
+    tensor-core sum is not correctly rounded), times scale * K: 2e-3 bounds
+    that with room, against gradient entries of size 0.1 to 1 otherwise."""
+    q, k, v = (t.cuda() for t in inputs.qkv(2, 3, 1, 128, seed=8))
+    do = inputs.grad_out(2, 3, 1, 128, seed=8).cuda()
+    o, lse = lib.fwd(q, k, v, causal=causal)
+    dq, dk, dv = lib.bwd(q, k, v, o, do, lse, causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(dv, do)
+    assert dq.abs().max().item() <= 2e-3 and dk.abs().max().item() <= 2e-3
+
+
+@pytest.mark.parametrize("d", [8, 40, 96, 120])
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dims_padded(lib, d, causal):
+    """Head dims below 128 that are not 64 or 128 run zero-padded."""
+    errs, _ = _run(lib, 1, 2, 333, d, causal, seed=d)
+    for what, e in errs:
+        _assert_ok(e, ("d", d, causal, what))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp16(lib, d, causal):
+    errs, _ = _run(lib, 2, 2, 300, d, causal, dtype=torch.float16, seed=9)
+    for what, e in errs:
+        _assert_ok(e, ("fp16", d, causal, what))
+
+
+def test_many_heads_wrap_the_persistent_grid(lib):
+    """More work units than SMs: every CTA runs several units."""
+    errs, _ = _run(lib, 3, 40, 256, 64, True, seed=3, heads=[(0, 0), (1, 17), (2, 39)])
+    for what, e in errs:
+        _assert_ok(e, what)
+
+
+def test_scale_other_than_inverse_sqrt_d(lib):
+    errs, _ = _run(lib, 1, 2, 200, 128, False, seed=4, scale=0.3)
+    for what, e in errs:
+        _assert_ok(e, ("scale 0.3", what))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_long_sequence_heads(lib, causal):
+    """N = 4096, d = 128: two heads of a four-head call, every entry."""
+    errs, _ = _run(lib, 1, 4, 4096, 128, causal, seed=11, heads=[(0, 0), (0, 3)])
+    for what, e in errs:
+        _assert_ok(e, ("4096", causal, what))
+
+
+def test_deterministic_and_workspace_contents_irrelevant(lib):
+    B, H, N, d = 2, 3, 700, 128
+    q, k, v = (t.cuda() for t in inputs.qkv(B, H, N, d, seed=21))
+    do = inputs.grad_out(B, H, N, d, seed=21).cuda()
+    o, lse = lib.fwd(q, k, v, causal=True)
+    ws = torch.full((lib.bwd_workspace_bytes(B, H, N),), 0xFF, dtype=torch.uint8, device="cuda")  # NaN floats
+    a = lib.bwd(q, k, v, o, do, lse, causal=True, workspace=ws)
+    b = lib.bwd(q, k, v, o, do, lse, causal=True)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_outputs_past_the_last_row_untouched(lib):
+    """dQ, dK, dV are written for rows < N only: guard rows after the tensor
+    (inside one allocation) keep their contents."""
+    B, H, N, d = 1, 1, 130, 64
+    q, k, v = (t.cuda() for t in inputs.qkv(B, H, N, d, seed=2))
+    do = inputs.grad_out(B, H, N, d, seed=2).cuda()
+    o, lse = lib.fwd(q, k, v)
+    outs = []
+    for _ in range(3):
+        buf = torch.full((B * H * N * d + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+        outs.append(buf)
+    views = [buf[:B * H * N * d].view(B, H, N, d) for buf in outs]
+    lib.bwd(q, k, v, o, do, lse, dq=views[0], dk=views[1], dv=views[2])
+    torch.cuda.synchronize()
+    for buf in outs:
+        assert torch.all(buf[B * H * N * d:] == 7.0)
+
+
+def test_bad_arguments_raise(lib):
+    x = torch.zeros(1, 1, 128, 256, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(1, 1, 128, dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.AttnError):
+        lib.bwd(x, x, x, x, x, lse)
+    y = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        lib.bwd(y, y, y, y, y, lse[..., :64])
