@@ -316,6 +316,27 @@ def run_ours(args, world, rank, local):
     ms_c = timed(step_c, max(3, args.steps // 2), args.warmup, world) / max(3, args.steps // 2)
     tf_c = flops(B, H, N, d, True) / (ms_c * 1e-3) / 1e12
 
+    # backward (attn_bwd: dQ, dK, dV from dO, O and LSE), same shape; the
+    # nominal count is five N x N x d products, 2.5x the forward's
+    dod = inputs.grad_out(B, H, N, d, seed=rank_seed(rank)).to(dev)
+    dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+    bwd_ms = {}
+    for causal, det in ((False, False), (True, False), (False, True)):
+        ws = torch.empty(binding.bwd_workspace_bytes(B, H, N, d, det), dtype=torch.uint8, device=dev)
+        o_b, lse_b = torch.empty_like(qd), torch.empty_like(lse)
+        binding.fwd(qd, kd, vd, causal=causal, out=o_b, lse=lse_b)
+
+        def step_bwd():
+            binding.bwd(qd, kd, vd, o_b, dod, lse_b, causal=causal, dq=dq, dk=dk, dv=dv, workspace=ws,
+                        deterministic=det)
+        nb = max(3, args.steps // 8)
+        bwd_ms[(causal, det)] = timed(step_bwd, nb, args.warmup, world) / nb
+        del o_b, lse_b, ws
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"backward kernel status {code} at {where}")
+    del dq, dk, dv, dod
+
     # FP8 variant: outlier inputs, Hadamard rotation of Q and K, 128 x d block scales
     qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank_seed(rank), outliers=True))
     signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
@@ -382,6 +403,15 @@ def run_ours(args, world, rank, local):
         "variants": {
             "bf16_causal": {"tflops": tf_c, "ms": ms_c,
                             "pct_of_spec_bf16_peak": 100 * tf_c / SPEC_BF16_TFLOPS},
+            "bf16_backward_noncausal": {"tflops": 2.5 * f_nc / (bwd_ms[(False, False)] * 1e-3) / 1e12,
+                                        "ms": bwd_ms[(False, False)], "kernels_per_call": 3,
+                                        "path": "fused, dQ by fp32 atomic adds"},
+            "bf16_backward_causal": {"tflops": 2.5 * flops(B, H, N, d, True) / (bwd_ms[(True, False)] * 1e-3) / 1e12,
+                                     "ms": bwd_ms[(True, False)], "kernels_per_call": 3,
+                                     "path": "fused, dQ by fp32 atomic adds"},
+            "bf16_backward_noncausal_deterministic": {
+                "tflops": 2.5 * f_nc / (bwd_ms[(False, True)] * 1e-3) / 1e12, "ms": bwd_ms[(False, True)],
+                "kernels_per_call": 2, "path": "dQ kernel then dK/dV kernel, no atomics"},
             "fp8_e4m3_hadamard_noncausal": {
                 "tflops": tf_8, "ms": ms_8, "pct_of_spec_fp8_peak": 100 * tf_8 / SPEC_FP8_TFLOPS,
                 "quant_ms_qkv": ms_q,

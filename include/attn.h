@@ -181,11 +181,13 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void
                                void* stream);
 
 /*
- * attn_bwd_workspace_bytes -- size of the workspace attn_bwd needs:
- * B * H * ceil(N / 128) * 256 * 4 bytes (two fp32 values per query row,
- * rows padded to whole 128-row tiles).  Returns 0 for sizes < 1.
+ * attn_bwd_workspace_bytes -- size of the workspace attn_bwd needs for these
+ * sizes and mode: B * H * ceil(N / 128) * 256 * 4 bytes of row statistics
+ * (two fp32 values per query row, rows padded to whole 128-row tiles), plus,
+ * when `deterministic` is 0, B * H * N * d * 4 bytes of fp32 dQ accumulator.
+ * Returns 0 for sizes < 1 or a mode other than 0 / 1.
  */
-size_t attn_bwd_workspace_bytes(int B, int H, int N);
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int deterministic);
 
 /*
  * attn_bwd -- 16-bit attention backward: the gradients of O with respect to
@@ -206,23 +208,30 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N);
  *   lse             : [B][H][N] fp32 (natural log), read only.
  *   dq, dk, dv      : [B][H][N][d] same dtype, written.
  *   workspace       : device memory of at least attn_bwd_workspace_bytes(B,
- *                     H, N) bytes, 16-byte aligned, owned by the caller; its
- *                     contents on entry do not matter and are overwritten
- *                     (row statistics passed between the two kernels).
+ *                     H, N, d, deterministic) bytes, 16-byte aligned, owned
+ *                     by the caller; its contents on entry do not matter
+ *                     and are overwritten.
  *   d               : a multiple of 8, at most 128 (64 and 128 natively,
  *                     others zero-padded); larger d returns
  *                     ATTN_ERR_UNSUPPORTED.
+ *   deterministic   : 0 -- fused path (three kernels): one pass over the key
+ *                     tiles computes dK, dV and dQ; dQ is summed over key
+ *                     tiles by fp32 atomic adds into the workspace, so its
+ *                     last bits may differ from run to run (dK, dV do not).
+ *                     1 -- two kernels (dQ, then dK/dV), no atomics, every
+ *                     output bit-reproducible; recomputes S and dP, so it
+ *                     does seven N x N x d products instead of five.
  *   B, H, N, scale, causal, dtype, stream: as for attn_fwd.
  * Rounding: scores, P, dP and accumulation are fp32; P and dS are rounded to
  * the input dtype before the products that use them; D is accumulated in
  * fp32 from the 16-bit dO and O; outputs are rounded to the input dtype.
- * Deterministic (no atomics): two kernels on `stream`, the first writing
- * dQ and the workspace, the second dK and dV.
+ * The "Results are deterministic" convention above holds for
+ * deterministic = 1 only.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
                        const float* lse, void* dq, void* dk, void* dv, void* workspace,
                        size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
-                       int dtype, void* stream);
+                       int deterministic, int dtype, void* stream);
 
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t s);

@@ -31,8 +31,9 @@ SIGNATURES = {
     "attn_debug_set_fault": (_I, [_I, _I]),
     "attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
     "attn_fwd_strided": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _F, _I, _I, _P]),
-    "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
-    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _I, _I,
+                      _P]),
 }
 
 
@@ -163,18 +164,19 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool 
     return o, (lse if return_lse else None)
 
 
-def bwd_workspace_bytes(B: int, H: int, N: int) -> int:
-    return int(load().attn_bwd_workspace_bytes(int(B), int(H), int(N)))
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int, deterministic: bool = False) -> int:
+    return int(load().attn_bwd_workspace_bytes(int(B), int(H), int(N), int(d), int(bool(deterministic))))
 
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
-        dq=None, dk=None, dv=None, workspace=None):
+        dq=None, dk=None, dv=None, workspace=None, deterministic: bool = False):
     """dQ, dK, dV of attention through ``attn_bwd`` on the current stream.
 
     q, k, v, o, do: contiguous CUDA tensors [B, H, N, d] of one 16-bit dtype
     (o and lse from :func:`fwd` with the same causal and scale); lse fp32
     [B, H, N].  ``workspace`` (uint8, at least :func:`bwd_workspace_bytes`)
-    is allocated here when not given.
+    is allocated here when not given.  ``deterministic`` selects the
+    two-kernel path without atomics (bit-reproducible dQ).
     """
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         if not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
@@ -190,13 +192,14 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
-    nbytes = bwd_workspace_bytes(B, H, N)
+    nbytes = bwd_workspace_bytes(B, H, N, d, deterministic)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
     code = load().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
                            _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                           B, H, N, d, scale, int(bool(causal)), dtype, _stream(q.device))
+                           B, H, N, d, scale, int(bool(causal)), int(bool(deterministic)), dtype,
+                           _stream(q.device))
     _check("attn_bwd", code)
     return dq, dk, dv
 

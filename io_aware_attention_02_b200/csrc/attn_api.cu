@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "bwd_fused_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
@@ -270,8 +271,48 @@ attn_status_t launch_bwd_c(const attn::BwdParams& p, int sm_count, int causal, c
   return causal ? launch_bwd<E, D, true>(p, sm_count, s) : launch_bwd<E, D, false>(p, sm_count, s);
 }
 
-size_t bwd_workspace_bytes(int B, int H, int N) {
+// Fused path: row statistics, then the fused kernel, then the dQ conversion.
+template <typename E, int D, bool CAUSAL>
+attn_status_t launch_bwd_fused(attn::BwdParams p, int sm_count, const void* o, const void* d_o,
+                               cudaStream_t stream) {
+  using Cfg = attn::FusedCfg<D>;
+  auto kf = attn::attn_bwd_fused_kernel<E, D, CAUSAL>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_done = true;
+  }
+  attn::attn_bwd_prep_kernel<E><<<p.BH * p.n_t, 256, 0, stream>>>(
+      static_cast<const E*>(o), static_cast<const E*>(d_o), p.lse, p.rows, p.dq_acc, p.N, p.n_t, p.d_out);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  p.n_units = p.BH * p.n_t;
+  const int grid = p.n_units < sm_count ? p.n_units : sm_count;
+  p.snake = CAUSAL ? 1 : 0;
+  p.order = (CAUSAL && p.n_t < grid) ? 1 : 0;
+  kf<<<grid, Cfg::kThreads, Cfg::kSmem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  const size_t n8 = static_cast<size_t>(p.BH) * p.N * p.d_out / 8;
+  attn::attn_bwd_dq_convert_kernel<E><<<sm_count * 4, 256, 0, stream>>>(p.dq_acc, static_cast<E*>(p.dq), n8,
+                                                                        p.scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename E, int D>
+attn_status_t launch_bwd_fused_c(const attn::BwdParams& p, int sm_count, int causal, const void* o,
+                                 const void* d_o, cudaStream_t s) {
+  return causal ? launch_bwd_fused<E, D, true>(p, sm_count, o, d_o, s)
+                : launch_bwd_fused<E, D, false>(p, sm_count, o, d_o, s);
+}
+
+size_t bwd_rows_bytes(int B, int H, int N) {
   return static_cast<size_t>(B) * H * ((N + 127) / 128) * 256 * sizeof(float);
+}
+
+size_t bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
+  size_t b = bwd_rows_bytes(B, H, N);
+  if (!deterministic) b += static_cast<size_t>(B) * H * N * d * sizeof(float);
+  return b;
 }
 
 }  // namespace
@@ -496,24 +537,25 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
 }
 
-extern "C" size_t attn_bwd_workspace_bytes(int B, int H, int N) {
-  if (B < 1 || H < 1 || N < 1) return 0;
-  return bwd_workspace_bytes(B, H, N);
+extern "C" size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || (deterministic != 0 && deterministic != 1)) return 0;
+  return bwd_workspace_bytes(B, H, N, d, deterministic);
 }
 
 extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                   const void* d_o, const float* lse, void* dq, void* dk, void* dv,
                                   void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
-                                  float scale, int causal, int dtype, void* stream) {
+                                  float scale, int causal, int deterministic, int dtype, void* stream) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || d_o == nullptr || lse == nullptr ||
       dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
     return ATTN_ERR_INVALID_ARG;
   attn_status_t r = common_checks(B, H, N, scale, causal);
   if (r != ATTN_OK) return r;
+  if (deterministic != 0 && deterministic != 1) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
   if (d > 128 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
-  if (workspace_bytes < bwd_workspace_bytes(B, H, N)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(B, H, N, d, deterministic)) return ATTN_ERR_INVALID_ARG;
   const void* p16[] = {q, k, v, o, d_o, dq, dk, dv, workspace};
   for (const void* x : p16)
     if (!aligned16(x)) return ATTN_ERR_MISALIGNED;
@@ -535,6 +577,8 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
   p.dv = dv;
   p.lse = lse;
   p.rows = static_cast<float*>(workspace);
+  p.dq_acc = deterministic ? nullptr
+                           : reinterpret_cast<float*>(static_cast<char*>(workspace) + bwd_rows_bytes(B, H, N));
   p.status = st->status;
   p.BH = B * H;
   p.H = H;
@@ -545,10 +589,18 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int dk_ = d <= 64 ? 64 : 128;
-  if (dtype == ATTN_BF16)
-    return dk_ == 64 ? launch_bwd_c<__nv_bfloat16, 64>(p, st->sm_count, causal, s)
-                     : launch_bwd_c<__nv_bfloat16, 128>(p, st->sm_count, causal, s);
-  return dk_ == 64 ? launch_bwd_c<__half, 64>(p, st->sm_count, causal, s)
-                   : launch_bwd_c<__half, 128>(p, st->sm_count, causal, s);
+  const bool bf = dtype == ATTN_BF16;
+  const bool d64 = d <= 64;
+  if (deterministic) {
+    if (bf)
+      return d64 ? launch_bwd_c<__nv_bfloat16, 64>(p, st->sm_count, causal, s)
+                 : launch_bwd_c<__nv_bfloat16, 128>(p, st->sm_count, causal, s);
+    return d64 ? launch_bwd_c<__half, 64>(p, st->sm_count, causal, s)
+               : launch_bwd_c<__half, 128>(p, st->sm_count, causal, s);
+  }
+  if (bf)
+    return d64 ? launch_bwd_fused_c<__nv_bfloat16, 64>(p, st->sm_count, causal, o, d_o, s)
+               : launch_bwd_fused_c<__nv_bfloat16, 128>(p, st->sm_count, causal, o, d_o, s);
+  return d64 ? launch_bwd_fused_c<__half, 64>(p, st->sm_count, causal, o, d_o, s)
+             : launch_bwd_fused_c<__half, 128>(p, st->sm_count, causal, o, d_o, s);
 }

@@ -1,0 +1,452 @@
+// Fused attention backward for sm_100a: one pass over the key tiles that
+// produces dK, dV and dQ together (five N x N x d products instead of the
+// seven of the two-kernel path), with dQ summed across key tiles by fp32
+// atomic adds.  Same gradients as bwd_sm100.cuh ("FlashAttention-3"
+// explainer, droidorbit.com, definition Softmax(Q K^T / sqrt(d)) V, chain
+// rule):
+//
+//   P = exp(scale * Q K^T - LSE),  dV = P^T dO,  dS = P * (dO V^T - D),
+//   dK = scale * dS^T Q,           dQ = scale * dS K,   D = rowsum(dO * O)
+//
+// Three launches:
+//   attn_bwd_prep_kernel   D and LSE * log2(e) per query row (row-statistics
+//                          workspace) and zeroes the fp32 dQ accumulator;
+//   attn_bwd_fused_kernel  one 128-key tile per work unit, all Q tiles it
+//                          meets;
+//   attn_bwd_dq_convert_kernel  dQ = scale * accumulator, rounded to 16 bits.
+//
+// Fused kernel, per Q tile i of the unit's key tile j (TMEM columns at d=128:
+// S^T 0-127 | dP^T 128-255 | dV 256-383 | dK 384-511):
+//   MMA   S^T = K Q_i^T, dP^T = V dO_i^T (SS, both K-major)
+//   rows  (warps 4-7, thread = key) P^T and dS^T, 16-bit, over S^T and dP^T
+//         in TMEM, and dS into shared memory (query-contiguous rows, the
+//         MN-major A operand of the dQ product)
+//   MMA   dV += P^T dO_i, dK += dS^T Q_i (TS), dQ_i = dS K_j (SS, both
+//         MN-major) into the dP^T columns, which dK has just consumed
+//   dQ    (warps 8-11, thread = query) TMEM -> fp32 atomic adds into the
+//         accumulator; the next dP^T waits for these loads only.
+// At d=64 dQ has columns of its own (384-447).  Every wait is bounded.
+#pragma once
+#include "bwd_sm100.cuh"
+
+namespace attn {
+
+template <int D>
+struct FusedCfg {
+  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (D == 64) ? 3 : 2;           // (Q, dO) ring
+  static constexpr int kRowBytes = 2 * 128 * 4;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffDS = kOffRing + kStages * 2 * kTileBytes;
+  static constexpr int kOffRow = kOffDS + 2 * kChunkBytes;    // dS: 128 keys x 128 queries, 16-bit
+  static constexpr int kOffBar = kOffRow + kStages * kRowBytes;
+  static constexpr int kSmem = kOffBar + 256;                  // base must be 1 KiB aligned (checked)
+  static constexpr int kThreads = 384;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr bool kDqShared = (D != 64);                 // dQ over the dP^T columns
+  static constexpr int kColDQ = kDqShared ? kColDP : 384;
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
+enum : int { kErrLayout = 4, kWhereLayout = 9 };
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO * O), LSE * log2(e) per row; dQ accumulator rows set to 0.
+// One 128-row tile per CTA of 256 threads, 16 threads per row (d <= 128).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const T* __restrict__ o, const T* __restrict__ d_o,
+                                                            const float* __restrict__ lse, float* rows,
+                                                            float* dq_acc, int N, int n_t, int d) {
+  const int tile = blockIdx.x;   // bh * n_t + q tile
+  const int bh = tile / n_t, qt = tile % n_t;
+  const int seg = threadIdx.x & 15;
+  float* out = rows + static_cast<size_t>(tile) * 256;
+  for (int rr = threadIdx.x >> 4; rr < 128; rr += 16) {
+    const int row = qt * 128 + rr;
+    const bool valid = row < N;
+    float dsum = 0.f;
+    if (valid && seg * 8 < d) {
+      const size_t off = (static_cast<size_t>(bh) * N + row) * d + seg * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(d_o + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(o + off);
+      const T* ta = reinterpret_cast<const T*>(&a);
+      const T* tb = reinterpret_cast<const T*>(&b);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dsum = fmaf(static_cast<float>(ta[e]), static_cast<float>(tb[e]), dsum);
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = 8; m >= 1; m >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
+    if (seg == 0) {
+      out[rr] = valid ? lse[static_cast<size_t>(bh) * N + row] * 1.4426950408889634f : 0.f;
+      out[128 + rr] = dsum;
+    }
+  }
+}
+
+// dq = scale * acc, eight elements per step.
+template <typename T>
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc, T* __restrict__ dq,
+                                                                  size_t n8, float scale) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    reinterpret_cast<uint4*>(dq)[i] = make_uint4(pack2<T>(a.x * scale, a.y * scale), pack2<T>(a.z * scale, a.w * scale),
+                                                 pack2<T>(b.x * scale, b.y * scale), pack2<T>(b.z * scale, b.w * scale));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The fused kernel
+// ---------------------------------------------------------------------------
+template <typename E, int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
+  using Cfg = FusedCfg<D>;
+  using T = E;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The layout fills the 227 KiB budget at d=128 with no room to realign.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) report_error(p.status, kErrLayout, kWhereLayout);
+    return;
+  }
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + Cfg::kOffV;
+  uint8_t* sRing = smem + Cfg::kOffRing;   // stage s: Q tile, then dO tile
+  uint8_t* sDS = smem + Cfg::kOffDS;
+  const float* sRows = reinterpret_cast<const float*>(smem + Cfg::kOffRow);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* sd_full = bars + 2;      // S^T, dP^T in TMEM
+  uint64_t* p_ready = bars + 3;      // P^T, dS^T in TMEM and dS in shared memory
+  uint64_t* dq_full = bars + 4;      // dQ_i in TMEM
+  uint64_t* dq_empty = bars + 5;     // dQ_i loaded out of TMEM
+  uint64_t* acc_full = bars + 6;     // dV, dK of the unit complete
+  uint64_t* drain = bars + 7;
+  uint64_t* q_full = bars + 8;       // [S]
+  uint64_t* q_empty = bars + 8 + S;  // [S]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * S);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
+  constexpr int kColDQ = Cfg::kColDQ;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(sd_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const unsigned long long lim = p.wait_limit_ns;
+  const int n_t = p.n_t;
+  auto key_tile = [&](int blk) { return CAUSAL ? n_t - 1 - blk : blk; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      uint32_t q_iter = 0, unit_iter = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh, blk;
+        decode_unit<CAUSAL>(unit, n_t, p.BH, p.order, bh, blk);
+        const int j = key_tile(blk);
+        const int i0 = CAUSAL ? j : 0;
+        const int h = bh % p.H, b = bh / p.H;
+        ok = mbar_wait(kv_empty, (unit_iter & 1) ^ 1, p.status, abort_flag, kWhereQEmpty, lim);
+        if (!ok) break;
+        mbar_arrive_expect_tx(kv_full, 2 * Cfg::kTileBytes);
+        for (int c = 0; c < Cfg::kChunks; ++c) {
+          tma_load_4d(sK + c * Cfg::kChunkBytes, &p.tm_k, kv_full, c * 64, j * 128, h, b);
+          tma_load_4d(sV + c * Cfg::kChunkBytes, &p.tm_v, kv_full, c * 64, j * 128, h, b);
+        }
+        for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
+          const uint32_t s = q_iter % S;
+          ok = mbar_wait(q_empty + s, ((q_iter / S) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
+          if (!ok) break;
+          mbar_arrive_expect_tx(q_full + s, 2 * Cfg::kTileBytes + Cfg::kRowBytes);
+          uint8_t* st = sRing + s * 2 * Cfg::kTileBytes;
+          for (int c = 0; c < Cfg::kChunks; ++c) {
+            tma_load_4d(st + c * Cfg::kChunkBytes, &p.tm_q, q_full + s, c * 64, i * 128, h, b);
+            tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_do, q_full + s, c * 64, i * 128, h, b);
+          }
+          bulk_load(smem + Cfg::kOffRow + s * Cfg::kRowBytes, p.rows + (static_cast<size_t>(bh) * n_t + i) * 256,
+                    Cfg::kRowBytes, q_full + s);
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        for (uint32_t i = (q_iter > S ? q_iter - S : 0); i < q_iter; ++i)
+          mbar_wait(q_full + (i % S), (i / S) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+        if (unit_iter > 0) mbar_wait(kv_full, (unit_iter - 1) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t fmt = Elem<E>::kFmt;
+      constexpr uint32_t idesc_kk = make_idesc(fmt, fmt, 0, 0, 128, 128);   // S^T, dP^T
+      constexpr uint32_t idesc_acc = make_idesc(fmt, fmt, 0, 1, 128, D);    // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t idesc_dq = make_idesc(fmt, fmt, 1, 1, 128, D);     // dQ: A, B MN-major
+      const uint64_t dKd = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dVd = smem_desc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), Cfg::kChunkBytes, 1024);
+      const uint64_t dDS = smem_desc_sw128(smem_u32(sDS), Cfg::kChunkBytes, 1024);
+      const uint64_t dRingK = smem_desc_sw128(smem_u32(sRing), 16, 1024);
+      const uint64_t dRingMN = smem_desc_sw128(smem_u32(sRing), Cfg::kChunkBytes, 1024);
+      uint32_t q_iter = 0, unit_iter = 0;
+      bool ok = true;
+      auto kmajor = [&](uint32_t d_col, uint64_t a0, uint64_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + d_col, a0 + off, b0 + off, idesc_kk, kk > 0, false);
+        }
+      };
+      auto accum = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + d_col, tmem + a_col + kk * 8, b0 + ((kk * 16 * 128) >> 4), idesc_acc,
+                 (acc || kk > 0) ? 1u : 0u, false);
+      };
+      // dQ may be overwritten once the previous tile's dQ has been loaded out
+      auto wait_dq_free = [&]() -> bool {
+        if (q_iter == 0) return true;
+        bool r = mbar_wait(dq_empty, (q_iter - 1) & 1, p.status, abort_flag, kWhereOFull, lim);
+        tc_fence_after();
+        return r;
+      };
+      for (int k = 0; ok; ++k, ++unit_iter) {
+        const int unit = sched_unit(k, p.snake);
+        if (unit >= p.n_units) break;
+        int bh_, blk;
+        decode_unit<CAUSAL>(unit, n_t, p.BH, p.order, bh_, blk);
+        (void)bh_;
+        const int j = key_tile(blk);
+        const int i0 = CAUSAL ? j : 0;
+        ok = mbar_wait(kv_full, unit_iter & 1, p.status, abort_flag, kWhereQFull, lim);
+        tc_fence_after();
+        if (!ok) break;
+        for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
+          const uint32_t s = q_iter % S;
+          if (!(ok = mbar_wait(q_full + s, (q_iter / S) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
+          tc_fence_after();
+          const uint32_t qoff = (s * 2 * Cfg::kTileBytes) >> 4, dooff = ((s * 2 + 1) * Cfg::kTileBytes) >> 4;
+          // S^T over P^T of the previous tile (consumed by the dV product
+          // issued before); dP^T over dS^T (consumed by dK) and, at d=128,
+          // over the previous dQ once it has been loaded out
+          kmajor(kColS, dKd, dRingK + qoff);
+          if (Cfg::kDqShared && !(ok = wait_dq_free())) break;
+          kmajor(kColDP, dVd, dRingK + dooff);
+          mma_commit(sd_full);
+          if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
+          tc_fence_after();
+          accum(kColDV, kColS, dRingMN + dooff, i > i0);   // dV += P^T dO_i
+          accum(kColDK, kColDP, dRingMN + qoff, i > i0);   // dK += dS^T Q_i
+          mma_commit(q_empty + s);
+          if (!Cfg::kDqShared && !(ok = wait_dq_free())) break;
+          // dQ_i = dS K_j: 16 keys (16 rows of 128 bytes in both operands) per product
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + kColDQ, dDS + ((kk * 16 * 128) >> 4), dKmn + ((kk * 16 * 128) >> 4), idesc_dq,
+                   kk > 0 ? 1u : 0u, false);
+          mma_commit(dq_full);
+        }
+        if (!ok) break;
+        mma_commit(acc_full);
+        mma_commit(kv_empty);
+      }
+      if (!ok) {
+        mma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, nullptr, &never, kWhereDrain, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------- key rows
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS;
+    const uint32_t tDP = tmem + lane_off + kColDP;
+    const float c2 = p.scale_log2;
+    uint8_t* ds_row = sDS + r * 128;
+    const int sw = r & 7;
+    uint32_t t = 0, acc_cnt = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int unit = sched_unit(k, p.snake);
+      if (unit >= p.n_units) break;
+      int bh, blk;
+      decode_unit<CAUSAL>(unit, n_t, p.BH, p.order, bh, blk);
+      const int j = key_tile(blk);
+      const int i0 = CAUSAL ? j : 0;
+      const int key = j * 128 + r;
+      const bool key_ok = key < p.N;
+      const size_t rbase = static_cast<size_t>(bh) * p.N;
+      for (int i = i0; i < n_t; ++i, ++t) {
+        const uint32_t s = t % S;
+        bool w = mbar_wait(q_full + s, (t / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
+        w = w && mbar_wait(sd_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+        tc_fence_after();
+        const float* lse2 = sRows + s * 256;
+        const float* dvec = lse2 + 128;
+        const int q0 = i * 128;
+        // every pair of this tile is visible: no per-element mask
+        const bool full = !(CAUSAL && i == j) && q0 + 128 <= p.N && j * 128 + 128 <= p.N;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS + cc * 32, sr);
+          tmem_ld32(tDP + cc * 32, dr);
+          tmem_wait_ld();
+          uint32_t pp[16], pd[16];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            // LSE2 and D of these 16 queries (broadcast shared-memory reads)
+            float lv[16], dv[16];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const float4 a = reinterpret_cast<const float4*>(lse2 + cc * 32 + hh * 16)[x];
+              const float4 b = reinterpret_cast<const float4*>(dvec + cc * 32 + hh * 16)[x];
+              lv[4 * x] = a.x; lv[4 * x + 1] = a.y; lv[4 * x + 2] = a.z; lv[4 * x + 3] = a.w;
+              dv[4 * x] = b.x; dv[4 * x + 1] = b.y; dv[4 * x + 2] = b.z; dv[4 * x + 3] = b.w;
+            }
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) {
+              float pv[2], dsv[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int x = hh * 16 + 2 * ii + e;   // column within the chunk
+                float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -lv[2 * ii + e]));
+                if (!full) {
+                  const int qg = q0 + cc * 32 + x;
+                  const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
+                  pr = vis ? pr : 0.f;
+                }
+                pv[e] = pr;
+                dsv[e] = pr * (__uint_as_float(dr[x]) - dv[2 * ii + e]);
+              }
+              pp[hh * 8 + ii] = pack2<T>(pv[0], pv[1]);
+              pd[hh * 8 + ii] = pack2<T>(dsv[0], dsv[1]);
+            }
+          }
+          tmem_st16(tS + cc * 16, pp);
+          tmem_st16(tDP + cc * 16, pd);
+          // dS row `key`, queries 32cc..32cc+31: 16-byte groups 4(cc%2)..+3 of
+          // chunk cc/2, 128-byte swizzled
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const int g = (cc & 1) * 4 + gg;
+            *reinterpret_cast<uint4*>(ds_row + (cc >> 1) * Cfg::kChunkBytes + ((g ^ sw) << 4)) =
+                make_uint4(pd[4 * gg], pd[4 * gg + 1], pd[4 * gg + 2], pd[4 * gg + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+      }
+      if (!ok) break;
+      bool w = mbar_wait(acc_full, acc_cnt & 1, p.status, abort_flag, kWhereOFull, lim);
+      ++acc_cnt;
+      if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+      tc_fence_after();
+      const size_t orow = (rbase + (key_ok ? key : 0)) * p.d_out;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tA = tmem + lane_off + (which == 0 ? kColDV : kColDK);
+        T* dst = reinterpret_cast<T*>(which == 0 ? p.dv : p.dk) + orow;
+        const float mul = which == 0 ? 1.0f : p.scale;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tA + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
+          tmem_wait_ld();
+          if (key_ok) store_row32<T>(dst, cc * 32, p.d_out, rr, mul);
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ rows
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t tDQ = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
+    uint32_t t = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int unit = sched_unit(k, p.snake);
+      if (unit >= p.n_units) break;
+      int bh, blk;
+      decode_unit<CAUSAL>(unit, n_t, p.BH, p.order, bh, blk);
+      const int j = key_tile(blk);
+      const int i0 = CAUSAL ? j : 0;
+      for (int i = i0; i < n_t; ++i, ++t) {
+        bool w = mbar_wait(dq_full, t & 1, p.status, abort_flag, kWhereDrain, lim);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+        tc_fence_after();
+        const int q = i * 128 + r;
+        const bool valid = q < p.N;
+        float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * p.d_out;
+        // 64 columns at a time; the MMA may reuse the columns once all are loaded
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          uint32_t rr[64];
+          tmem_ld32(tDQ + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(rr));
+          tmem_ld32(tDQ + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
+          tmem_wait_ld();
+          if (hh == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(dq_empty);
+          }
+          if (valid) {
+#pragma unroll
+            for (int g = 0; g < 16; ++g)
+              if (hh * 64 + 4 * g < p.d_out)
+                red_add_v4(acc + hh * 64 + 4 * g, __uint_as_float(rr[4 * g]), __uint_as_float(rr[4 * g + 1]),
+                           __uint_as_float(rr[4 * g + 2]), __uint_as_float(rr[4 * g + 3]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+}  // namespace attn

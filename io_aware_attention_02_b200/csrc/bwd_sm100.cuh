@@ -39,6 +39,7 @@ struct BwdParams {
   void* dv;
   const float* lse;                            // [BH][N] natural-log LSE of the forward
   float* rows;                                 // [BH][n_t][2][128]: LSE*log2(e) | D per Q tile
+  float* dq_acc;                               // [BH][N][d_out] fp32 dQ / scale (fused path)
   int* status;
   int BH, H, N, n_t, n_units, d_out;
   float scale, scale_log2;

@@ -109,22 +109,27 @@ def test_strided_validation(lib):
 
 
 def test_bwd_workspace_size(lib):
-    # two fp32 values per query row, rows padded to whole 128-row tiles
-    assert lib.attn_bwd_workspace_bytes(2, 3, 1) == 2 * 3 * 1 * 256 * 4
-    assert lib.attn_bwd_workspace_bytes(1, 1, 129) == 2 * 256 * 4
-    assert lib.attn_bwd_workspace_bytes(1, 1, 0) == 0
+    # two fp32 values per query row, rows padded to whole 128-row tiles, and
+    # (fused mode) an fp32 dQ accumulator
+    assert lib.attn_bwd_workspace_bytes(2, 3, 1, 64, 1) == 2 * 3 * 1 * 256 * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 129, 64, 1) == 2 * 256 * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 129, 64, 0) == 2 * 256 * 4 + 129 * 64 * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 0, 64, 0) == 0
+    assert lib.attn_bwd_workspace_bytes(1, 1, 8, 64, 2) == 0
 
 
-def test_bwd_validation(lib):
+@pytest.mark.parametrize("det", [0, 1])
+def test_bwd_validation(lib, det):
     F = lib.attn_bwd
-    ws = lib.attn_bwd_workspace_bytes(1, 2, 256)
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 256, 64, det)
 
     def call(**kw):
         a = dict(q=GOOD, k=GOOD, v=GOOD, o=GOOD, do=GOOD, lse=GOOD, dq=GOOD, dk=GOOD, dv=GOOD,
-                 ws=GOOD, ws_bytes=ws, B=1, H=2, N=256, d=64, scale=0.125, causal=0, dtype=0)
+                 ws=GOOD, ws_bytes=ws, B=1, H=2, N=256, d=64, scale=0.125, causal=0, det=det, dtype=0)
         a.update(kw)
         return F(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"], a["ws"],
-                 a["ws_bytes"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["dtype"], None)
+                 a["ws_bytes"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["det"], a["dtype"],
+                 None)
 
     assert call(lse=None) == binding.ATTN_ERR_INVALID_ARG
     assert call(ws=None) == binding.ATTN_ERR_INVALID_ARG
@@ -132,6 +137,7 @@ def test_bwd_validation(lib):
     assert call(ws_bytes=ws - 4) == binding.ATTN_ERR_INVALID_ARG
     assert call(N=0) == binding.ATTN_ERR_INVALID_ARG
     assert call(causal=3) == binding.ATTN_ERR_INVALID_ARG
+    assert call(det=2) == binding.ATTN_ERR_INVALID_ARG
     assert call(d=256) == binding.ATTN_ERR_UNSUPPORTED
     assert call(d=100) == binding.ATTN_ERR_UNSUPPORTED
     assert call(dtype=2) == binding.ATTN_ERR_UNSUPPORTED
