@@ -103,6 +103,21 @@ attn_status_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType d
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// 3-D fp32 map over the backward's dQ accumulator [BH][N][d]: box 32 x 32
+// rows, 128-byte swizzle (reduce-add target; rows past N are not written).
+attn_status_t make_map_dq(CUtensorMap* map, float* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return ATTN_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(N) * d * 4};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 unsigned long long wait_limit_ns() {
   static unsigned long long ns = [] {
     const char* e = std::getenv("ATTN_WAIT_LIMIT_MS");
@@ -579,6 +594,7 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
   p.rows = static_cast<float*>(workspace);
   p.dq_acc = deterministic ? nullptr
                            : reinterpret_cast<float*>(static_cast<char*>(workspace) + bwd_rows_bytes(B, H, N));
+  if (!deterministic && (r = make_map_dq(&p.tm_dq, p.dq_acc, B * H, N, d)) != ATTN_OK) return r;
   p.status = st->status;
   p.BH = B * H;
   p.H = H;

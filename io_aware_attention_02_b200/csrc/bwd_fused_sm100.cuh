@@ -18,13 +18,16 @@
 // Fused kernel, per Q tile i of the unit's key tile j (TMEM columns at d=128:
 // S^T 0-127 | dP^T 128-255 | dV 256-383 | dK 384-511):
 //   MMA   S^T = K Q_i^T, dP^T = V dO_i^T (SS, both K-major)
-//   rows  (warps 4-7, thread = key) P^T and dS^T, 16-bit, over S^T and dP^T
-//         in TMEM, and dS into shared memory (query-contiguous rows, the
-//         MN-major A operand of the dQ product)
+//   rows  two warpgroups, thread = key, queries 0-63 and 64-127: P^T and
+//         dS^T, 16-bit, packed into TMEM columns 32-95 of S^T and dP^T (each
+//         warpgroup writes only columns it has already read), and dS into
+//         shared memory (query-contiguous rows, the MN-major A operand of the
+//         dQ product)
 //   MMA   dV += P^T dO_i, dK += dS^T Q_i (TS), dQ_i = dS K_j (SS, both
 //         MN-major) into the dP^T columns, which dK has just consumed
-//   dQ    (warps 8-11, thread = query) TMEM -> fp32 atomic adds into the
-//         accumulator; the next dP^T waits for these loads only.
+//   dQ    one warpgroup, thread = query: TMEM -> registers (the next dP^T
+//         may then start), then 32 x 32 fp32 boxes staged through the dS
+//         buffer and added into the accumulator by TMA reduce-add.
 // At d=64 dQ has columns of its own (384-447).  Every wait is bounded.
 #pragma once
 #include "bwd_sm100.cuh"
@@ -44,7 +47,7 @@ struct FusedCfg {
   static constexpr int kOffRow = kOffDS + 2 * kChunkBytes;    // dS: 128 keys x 128 queries, 16-bit
   static constexpr int kOffBar = kOffRow + kStages * kRowBytes;
   static constexpr int kSmem = kOffBar + 256;                  // base must be 1 KiB aligned (checked)
-  static constexpr int kThreads = 384;
+  static constexpr int kThreads = 512;
   static constexpr int kTmemCols = 512;
   static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr bool kDqShared = (D != 64);                 // dQ over the dP^T columns
@@ -107,8 +110,15 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
 // ---------------------------------------------------------------------------
 // The fused kernel
 // ---------------------------------------------------------------------------
+// Register split (setmaxnreg, per warpgroup): 512 threads launch with 128
+// registers each; the TMA/MMA warpgroup keeps 104 and gives the rest to the
+// two row warpgroups and the dQ warpgroup (104 + 3 * 136 = 4 * 128).
+constexpr int kBwdRegsLow = 104;
+constexpr int kBwdRegsHigh = 136;
+static_assert(128 * kBwdRegsLow + 384 * kBwdRegsHigh <= 512 * 128, "register split exceeds the launch pool");
+
 template <typename E, int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
   using Cfg = FusedCfg<D>;
   using T = E;
   constexpr int S = Cfg::kStages;
@@ -121,7 +131,7 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
   uint8_t* sK = smem;
   uint8_t* sV = smem + Cfg::kOffV;
   uint8_t* sRing = smem + Cfg::kOffRing;   // stage s: Q tile, then dO tile
-  uint8_t* sDS = smem + Cfg::kOffDS;
+  uint8_t* sDS = smem + Cfg::kOffDS;       // dS (MMA operand), then dQ staging
   const float* sRows = reinterpret_cast<const float*>(smem + Cfg::kOffRow);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* kv_full = bars + 0;
@@ -130,14 +140,16 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
   uint64_t* p_ready = bars + 3;      // P^T, dS^T in TMEM and dS in shared memory
   uint64_t* dq_full = bars + 4;      // dQ_i in TMEM
   uint64_t* dq_empty = bars + 5;     // dQ_i loaded out of TMEM
-  uint64_t* acc_full = bars + 6;     // dV, dK of the unit complete
-  uint64_t* drain = bars + 7;
-  uint64_t* q_full = bars + 8;       // [S]
-  uint64_t* q_empty = bars + 8 + S;  // [S]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * S);
+  uint64_t* ds_free = bars + 6;      // dQ_i staging read by TMA: the dS buffer is free
+  uint64_t* acc_full = bars + 7;     // dV, dK of the unit complete
+  uint64_t* drain = bars + 8;
+  uint64_t* q_full = bars + 9;       // [S]
+  uint64_t* q_empty = bars + 9 + S;  // [S]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * S);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
   constexpr int kColDQ = Cfg::kColDQ;
+  constexpr int kPk = 32;            // packed P^T / dS^T start 32 columns into S^T / dP^T
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -145,9 +157,10 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
     mbar_init(sd_full, 1);
-    mbar_init(p_ready, 128);
+    mbar_init(p_ready, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
+    mbar_init(ds_free, 4);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     for (int s = 0; s < S; ++s) {
@@ -169,6 +182,8 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
   const int n_t = p.n_t;
   auto key_tile = [&](int blk) { return CAUSAL ? n_t - 1 - blk : blk; };
 
+  if (warp < 4) {
+  reg_dealloc<kBwdRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -233,6 +248,7 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
           mma_ss(tmem + d_col, a0 + off, b0 + off, idesc_kk, kk > 0, false);
         }
       };
+      // A = 128 keys x 128 queries, 16-bit packed from column a_col (8 columns per 16 queries)
       auto accum = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -271,8 +287,8 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
           mma_commit(sd_full);
           if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
           tc_fence_after();
-          accum(kColDV, kColS, dRingMN + dooff, i > i0);   // dV += P^T dO_i
-          accum(kColDK, kColDP, dRingMN + qoff, i > i0);   // dK += dS^T Q_i
+          accum(kColDV, kColS + kPk, dRingMN + dooff, i > i0);   // dV += P^T dO_i
+          accum(kColDK, kColDP + kPk, dRingMN + qoff, i > i0);   // dK += dS^T Q_i
           mma_commit(q_empty + s);
           if (!Cfg::kDqShared && !(ok = wait_dq_free())) break;
           // dQ_i = dS K_j: 16 keys (16 rows of 128 bytes in both operands) per product
@@ -293,15 +309,18 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+  }
+  } else if (warp < 12) {
+    reg_alloc<kBwdRegsHigh>();
     // ------------------------------------------------------------- key rows
+    const int half = (warp - 4) >> 2;          // queries 64*half .. 64*half+63
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS;
     const uint32_t tDP = tmem + lane_off + kColDP;
     const float c2 = p.scale_log2;
-    uint8_t* ds_row = sDS + r * 128;
+    uint8_t* ds_row = sDS + half * Cfg::kChunkBytes + r * 128;
     const int sw = r & 7;
     uint32_t t = 0, acc_cnt = 0;
     bool ok = true;
@@ -319,6 +338,8 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
         const uint32_t s = t % S;
         bool w = mbar_wait(q_full + s, (t / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
         w = w && mbar_wait(sd_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
+        // the dS buffer: free once the previous tile's dQ staging has been read
+        w = w && (t == 0 || mbar_wait(ds_free, (t - 1) & 1, p.status, abort_flag, kWhereDrain, lim));
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
         const float* lse2 = sRows + s * 256;
@@ -326,51 +347,51 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
         const int q0 = i * 128;
         // every pair of this tile is visible: no per-element mask
         const bool full = !(CAUSAL && i == j) && q0 + 128 <= p.N && j * 128 + 128 <= p.N;
+        // Chunks of 32 queries, in an order that makes every packed write
+        // land on columns this warpgroup has already read: half 0 reads
+        // 0-63 and writes 32-63 (chunk 1 first), half 1 reads 64-127 and
+        // writes 64-95.
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int n = 0; n < 2; ++n) {
+          const int cc = half == 0 ? 1 - n : 2 + n;
           uint32_t sr[32], dr[32];
           tmem_ld32(tS + cc * 32, sr);
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
           uint32_t pp[16], pd[16];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            // LSE2 and D of these 16 queries (broadcast shared-memory reads)
-            float lv[16], dv[16];
+          for (int x4 = 0; x4 < 8; ++x4) {
+            // LSE2 and D of 4 queries (broadcast shared-memory reads)
+            const float4 lv = reinterpret_cast<const float4*>(lse2 + cc * 32)[x4];
+            const float4 dv = reinterpret_cast<const float4*>(dvec + cc * 32)[x4];
+            const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+            const float d4[4] = {dv.x, dv.y, dv.z, dv.w};
+            float pv[4], dsv[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const float4 a = reinterpret_cast<const float4*>(lse2 + cc * 32 + hh * 16)[x];
-              const float4 b = reinterpret_cast<const float4*>(dvec + cc * 32 + hh * 16)[x];
-              lv[4 * x] = a.x; lv[4 * x + 1] = a.y; lv[4 * x + 2] = a.z; lv[4 * x + 3] = a.w;
-              dv[4 * x] = b.x; dv[4 * x + 1] = b.y; dv[4 * x + 2] = b.z; dv[4 * x + 3] = b.w;
-            }
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii) {
-              float pv[2], dsv[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int x = hh * 16 + 2 * ii + e;   // column within the chunk
-                float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -lv[2 * ii + e]));
-                if (!full) {
-                  const int qg = q0 + cc * 32 + x;
-                  const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
-                  pr = vis ? pr : 0.f;
-                }
-                pv[e] = pr;
-                dsv[e] = pr * (__uint_as_float(dr[x]) - dv[2 * ii + e]);
+            for (int e = 0; e < 4; ++e) {
+              const int x = 4 * x4 + e;
+              float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -l4[e]));
+              if (!full) {
+                const int qg = q0 + cc * 32 + x;
+                const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
+                pr = vis ? pr : 0.f;
               }
-              pp[hh * 8 + ii] = pack2<T>(pv[0], pv[1]);
-              pd[hh * 8 + ii] = pack2<T>(dsv[0], dsv[1]);
+              pv[e] = pr;
+              dsv[e] = pr * (__uint_as_float(dr[x]) - d4[e]);
             }
+            pp[2 * x4] = pack2<T>(pv[0], pv[1]);
+            pp[2 * x4 + 1] = pack2<T>(pv[2], pv[3]);
+            pd[2 * x4] = pack2<T>(dsv[0], dsv[1]);
+            pd[2 * x4 + 1] = pack2<T>(dsv[2], dsv[3]);
           }
-          tmem_st16(tS + cc * 16, pp);
-          tmem_st16(tDP + cc * 16, pd);
+          tmem_st16(tS + kPk + cc * 16, pp);
+          tmem_st16(tDP + kPk + cc * 16, pd);
           // dS row `key`, queries 32cc..32cc+31: 16-byte groups 4(cc%2)..+3 of
-          // chunk cc/2, 128-byte swizzled
+          // this half's chunk, 128-byte swizzled
 #pragma unroll
           for (int gg = 0; gg < 4; ++gg) {
             const int g = (cc & 1) * 4 + gg;
-            *reinterpret_cast<uint4*>(ds_row + (cc >> 1) * Cfg::kChunkBytes + ((g ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(ds_row + ((g ^ sw) << 4)) =
                 make_uint4(pd[4 * gg], pd[4 * gg + 1], pd[4 * gg + 2], pd[4 * gg + 3]);
           }
         }
@@ -384,26 +405,26 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
       ++acc_cnt;
       if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
       tc_fence_after();
-      const size_t orow = (rbase + (key_ok ? key : 0)) * p.d_out;
+      // half 0 stores dV, half 1 stores dK (times scale)
+      const uint32_t tA = tmem + lane_off + (half == 0 ? kColDV : kColDK);
+      T* dst = reinterpret_cast<T*>(half == 0 ? p.dv : p.dk) + (rbase + (key_ok ? key : 0)) * p.d_out;
+      const float mul = half == 0 ? 1.0f : p.scale;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tA = tmem + lane_off + (which == 0 ? kColDV : kColDK);
-        T* dst = reinterpret_cast<T*>(which == 0 ? p.dv : p.dk) + orow;
-        const float mul = which == 0 ? 1.0f : p.scale;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t rr[32];
-          tmem_ld32(tA + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
-          tmem_wait_ld();
-          if (key_ok) store_row32<T>(dst, cc * 32, p.d_out, rr, mul);
-        }
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t rr[32];
+        tmem_ld32(tA + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
+        tmem_wait_ld();
+        if (key_ok) store_row32<T>(dst, cc * 32, p.d_out, rr, mul);
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    reg_alloc<kBwdRegsHigh>();
     // ------------------------------------------------------------ dQ rows
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
+    const int quarter = warp & 3;              // rows 32*quarter .. +31 of the Q tile
     const uint32_t tDQ = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
+    constexpr int kStageBytes = 16384;                   // one box buffer: 4 warps x 32 rows x 128 bytes
+    uint8_t* stage = sDS + quarter * 4096 + lane * 128;   // this lane's row in box buffer 0
+    const int sw = lane & 7;
     uint32_t t = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -417,10 +438,9 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
         bool w = mbar_wait(dq_full, t & 1, p.status, abort_flag, kWhereDrain, lim);
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
-        const int q = i * 128 + r;
-        const bool valid = q < p.N;
-        float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * p.d_out;
-        // 64 columns at a time; the MMA may reuse the columns once all are loaded
+        // 64 columns at a time: load, stage as two 32 x 32 boxes, reduce-add.
+        // dq_empty is signalled once every column has been loaded.
+        const int row0 = i * 128 + quarter * 32;
 #pragma unroll
         for (int hh = 0; hh < D / 64; ++hh) {
           uint32_t rr[64];
@@ -431,16 +451,37 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_fused_kernel(const __grid_con
             tc_fence_before();
             mbar_arrive(dq_empty);
           }
-          if (valid) {
 #pragma unroll
-            for (int g = 0; g < 16; ++g)
-              if (hh * 64 + 4 * g < p.d_out)
-                red_add_v4(acc + hh * 64 + 4 * g, __uint_as_float(rr[4 * g]), __uint_as_float(rr[4 * g + 1]),
-                           __uint_as_float(rr[4 * g + 2]), __uint_as_float(rr[4 * g + 3]));
+          for (int mm = 0; mm < 2; ++mm) {
+            const int m = 2 * hh + mm;   // box: columns 32m .. 32m+31, buffer m % 2
+            if (m >= 2) {
+              if (lane == 0) bulk_wait_group_read<1>();   // box m-2 has left this buffer
+              __syncwarp();
+            }
+            uint8_t* dst = stage + mm * kStageBytes;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              *reinterpret_cast<uint4*>(dst + ((g ^ sw) << 4)) =
+                  make_uint4(rr[32 * mm + 4 * g], rr[32 * mm + 4 * g + 1], rr[32 * mm + 4 * g + 2],
+                             rr[32 * mm + 4 * g + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < p.N && 32 * m < p.d_out)
+                tma_reduce_add_3d(&p.tm_dq, sDS + mm * kStageBytes + quarter * 4096, 32 * m, row0, bh);
+              bulk_commit_group();
+            }
           }
         }
+        if (lane == 0) {
+          bulk_wait_group_read<0>();
+          mbar_arrive(ds_free);
+        }
+        __syncwarp();
       }
     }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -34,6 +34,7 @@ namespace attn {
 
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_o, tm_do;   // 4-D maps (d, N, H, B), 64-column boxes
+  CUtensorMap tm_dq;                           // fp32 accumulator (d, N, BH), 32 x 32 boxes (fused path)
   void* dq;                                    // [BH][N][d_out] 16-bit outputs
   void* dk;
   void* dv;
