@@ -26,8 +26,10 @@
 //   MMA   dV += P^T dO_i, dK += dS^T Q_i (TS), dQ_i = dS K_j (SS, both
 //         MN-major) into the dP^T columns, which dK has just consumed
 //   dQ    one warpgroup, thread = query: TMEM -> registers (the next dP^T
-//         may then start), then 32 x 32 fp32 boxes staged through the dS
-//         buffer and added into the accumulator by TMA reduce-add.
+//         may then start), then 32 x 32 fp32 boxes staged in shared memory
+//         and added into the accumulator by TMA reduce-add.
+// Shared memory at d=128: K, V, two Q stages, one dO buffer (released right
+// after the dV product), dS, two dQ staging buffers: 7 x 32 KiB.
 // At d=64 dQ has columns of its own (384-447).  Every wait is bounded.
 #pragma once
 #include "bwd_sm100.cuh"
@@ -39,13 +41,17 @@ struct FusedCfg {
   static constexpr int kChunkBytes = 128 * 128;
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 64) ? 3 : 2;           // (Q, dO) ring
+  static constexpr int kQStages = (D == 64) ? 3 : 2;          // Q ring (with the row statistics)
+  static constexpr int kDoStages = (D == 64) ? 2 : 1;         // dO ring: released right after dV
   static constexpr int kRowBytes = 2 * 128 * 4;
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffRing = 2 * kTileBytes;
-  static constexpr int kOffDS = kOffRing + kStages * 2 * kTileBytes;
-  static constexpr int kOffRow = kOffDS + 2 * kChunkBytes;    // dS: 128 keys x 128 queries, 16-bit
-  static constexpr int kOffBar = kOffRow + kStages * kRowBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;
+  static constexpr int kOffDo = kOffQ + kQStages * kTileBytes;
+  static constexpr int kOffDS = kOffDo + kDoStages * kTileBytes;    // dS: 128 keys x 128 queries, 16-bit
+  static constexpr int kOffStage = kOffDS + 2 * kChunkBytes;       // dQ staging: two 16 KiB box buffers
+  static constexpr int kStageBytes = kChunkBytes;
+  static constexpr int kOffRow = kOffStage + 2 * kStageBytes;
+  static constexpr int kOffBar = kOffRow + kQStages * kRowBytes;
   static constexpr int kSmem = kOffBar + 256;                  // base must be 1 KiB aligned (checked)
   static constexpr int kThreads = 512;
   static constexpr int kTmemCols = 512;
@@ -111,17 +117,17 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
 // The fused kernel
 // ---------------------------------------------------------------------------
 // Register split (setmaxnreg, per warpgroup): 512 threads launch with 128
-// registers each; the TMA/MMA warpgroup keeps 104 and gives the rest to the
-// two row warpgroups and the dQ warpgroup (104 + 3 * 136 = 4 * 128).
-constexpr int kBwdRegsLow = 104;
-constexpr int kBwdRegsHigh = 136;
-static_assert(128 * kBwdRegsLow + 384 * kBwdRegsHigh <= 512 * 128, "register split exceeds the launch pool");
+// registers each; the TMA/MMA warpgroup gives 32 to the dQ warpgroup, which
+// holds a whole 128-column dQ tile (96 + 128 + 128 + 160 = 4 * 128).
+constexpr int kBwdRegsLow = 96;
+constexpr int kBwdRegsDq = 160;
+static_assert(128 * kBwdRegsLow + 256 * 128 + 128 * kBwdRegsDq <= 512 * 128, "register split exceeds the launch pool");
 
 template <typename E, int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
   using Cfg = FusedCfg<D>;
   using T = E;
-  constexpr int S = Cfg::kStages;
+  constexpr int SQ = Cfg::kQStages, SD = Cfg::kDoStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The layout fills the 227 KiB budget at d=128 with no room to realign.
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -130,8 +136,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   }
   uint8_t* sK = smem;
   uint8_t* sV = smem + Cfg::kOffV;
-  uint8_t* sRing = smem + Cfg::kOffRing;   // stage s: Q tile, then dO tile
-  uint8_t* sDS = smem + Cfg::kOffDS;       // dS (MMA operand), then dQ staging
+  uint8_t* sQ = smem + Cfg::kOffQ;
+  uint8_t* sDo = smem + Cfg::kOffDo;
+  uint8_t* sDS = smem + Cfg::kOffDS;       // dS, the A operand of the dQ product
+  uint8_t* sStage = smem + Cfg::kOffStage;
   const float* sRows = reinterpret_cast<const float*>(smem + Cfg::kOffRow);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* kv_full = bars + 0;
@@ -140,12 +148,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   uint64_t* p_ready = bars + 3;      // P^T, dS^T in TMEM and dS in shared memory
   uint64_t* dq_full = bars + 4;      // dQ_i in TMEM
   uint64_t* dq_empty = bars + 5;     // dQ_i loaded out of TMEM
-  uint64_t* ds_free = bars + 6;      // dQ_i staging read by TMA: the dS buffer is free
-  uint64_t* acc_full = bars + 7;     // dV, dK of the unit complete
-  uint64_t* drain = bars + 8;
-  uint64_t* q_full = bars + 9;       // [S]
-  uint64_t* q_empty = bars + 9 + S;  // [S]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * S);
+  uint64_t* acc_full = bars + 6;     // dV, dK of the unit complete
+  uint64_t* drain = bars + 7;
+  uint64_t* q_full = bars + 8;                 // [SQ] Q tile and its row statistics
+  uint64_t* q_empty = bars + 8 + SQ;           // [SQ]
+  uint64_t* do_full = bars + 8 + 2 * SQ;       // [SD]
+  uint64_t* do_empty = bars + 8 + 2 * SQ + SD; // [SD]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * SQ + 2 * SD);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
   constexpr int kColDQ = Cfg::kColDQ;
@@ -160,12 +169,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
     mbar_init(p_ready, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
-    mbar_init(ds_free, 4);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SQ; ++s) {
       mbar_init(q_full + s, 1);
       mbar_init(q_empty + s, 1);
+    }
+    for (int s = 0; s < SD; ++s) {
+      mbar_init(do_full + s, 1);
+      mbar_init(do_empty + s, 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -187,7 +199,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
-      uint32_t q_iter = 0, unit_iter = 0;
+      uint32_t nq = 0, nd = 0, unit_iter = 0;   // Q and dO tiles issued, units started
       bool ok = true;
       for (int k = 0; ok; ++k, ++unit_iter) {
         const int unit = sched_unit(k, p.snake);
@@ -204,24 +216,32 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           tma_load_4d(sK + c * Cfg::kChunkBytes, &p.tm_k, kv_full, c * 64, j * 128, h, b);
           tma_load_4d(sV + c * Cfg::kChunkBytes, &p.tm_v, kv_full, c * 64, j * 128, h, b);
         }
-        for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
-          const uint32_t s = q_iter % S;
-          ok = mbar_wait(q_empty + s, ((q_iter / S) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
+        for (int i = i0; i < n_t && ok; ++i) {
+          const uint32_t sq = nq % SQ;
+          ok = mbar_wait(q_empty + sq, ((nq / SQ) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
           if (!ok) break;
-          mbar_arrive_expect_tx(q_full + s, 2 * Cfg::kTileBytes + Cfg::kRowBytes);
-          uint8_t* st = sRing + s * 2 * Cfg::kTileBytes;
-          for (int c = 0; c < Cfg::kChunks; ++c) {
-            tma_load_4d(st + c * Cfg::kChunkBytes, &p.tm_q, q_full + s, c * 64, i * 128, h, b);
-            tma_load_4d(st + Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_do, q_full + s, c * 64, i * 128, h, b);
-          }
-          bulk_load(smem + Cfg::kOffRow + s * Cfg::kRowBytes, p.rows + (static_cast<size_t>(bh) * n_t + i) * 256,
-                    Cfg::kRowBytes, q_full + s);
+          mbar_arrive_expect_tx(q_full + sq, Cfg::kTileBytes + Cfg::kRowBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sQ + sq * Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_q, q_full + sq, c * 64, i * 128, h, b);
+          bulk_load(smem + Cfg::kOffRow + sq * Cfg::kRowBytes, p.rows + (static_cast<size_t>(bh) * n_t + i) * 256,
+                    Cfg::kRowBytes, q_full + sq);
+          ++nq;
+          const uint32_t sd = nd % SD;
+          ok = mbar_wait(do_empty + sd, ((nd / SD) & 1) ^ 1, p.status, abort_flag, kWhereKvEmpty, lim);
+          if (!ok) break;
+          mbar_arrive_expect_tx(do_full + sd, Cfg::kTileBytes);
+          for (int c = 0; c < Cfg::kChunks; ++c)
+            tma_load_4d(sDo + sd * Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_do, do_full + sd, c * 64, i * 128, h, b);
+          ++nd;
         }
       }
       if (!ok) {
+        // let the copies already issued land before the CTA exits
         volatile int never = 0;
-        for (uint32_t i = (q_iter > S ? q_iter - S : 0); i < q_iter; ++i)
-          mbar_wait(q_full + (i % S), (i / S) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+        for (uint32_t i = (nq > SQ ? nq - SQ : 0); i < nq; ++i)
+          mbar_wait(q_full + (i % SQ), (i / SQ) & 1, nullptr, &never, kWhereDrain, 100000000ull);
+        for (uint32_t i = (nd > SD ? nd - SD : 0); i < nd; ++i)
+          mbar_wait(do_full + (i % SD), (i / SD) & 1, nullptr, &never, kWhereDrain, 100000000ull);
         if (unit_iter > 0) mbar_wait(kv_full, (unit_iter - 1) & 1, nullptr, &never, kWhereDrain, 100000000ull);
       }
     }
@@ -237,8 +257,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
       const uint64_t dVd = smem_desc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dKmn = smem_desc_sw128(smem_u32(sK), Cfg::kChunkBytes, 1024);
       const uint64_t dDS = smem_desc_sw128(smem_u32(sDS), Cfg::kChunkBytes, 1024);
-      const uint64_t dRingK = smem_desc_sw128(smem_u32(sRing), 16, 1024);
-      const uint64_t dRingMN = smem_desc_sw128(smem_u32(sRing), Cfg::kChunkBytes, 1024);
+      const uint64_t dQk = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dQmn = smem_desc_sw128(smem_u32(sQ), Cfg::kChunkBytes, 1024);
+      const uint64_t dDok = smem_desc_sw128(smem_u32(sDo), 16, 1024);
+      const uint64_t dDomn = smem_desc_sw128(smem_u32(sDo), Cfg::kChunkBytes, 1024);
       uint32_t q_iter = 0, unit_iter = 0;
       bool ok = true;
       auto kmajor = [&](uint32_t d_col, uint64_t a0, uint64_t b0) {
@@ -274,22 +296,25 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         tc_fence_after();
         if (!ok) break;
         for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
-          const uint32_t s = q_iter % S;
-          if (!(ok = mbar_wait(q_full + s, (q_iter / S) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
+          const uint32_t sq = q_iter % SQ, sd = q_iter % SD;
+          if (!(ok = mbar_wait(q_full + sq, (q_iter / SQ) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
           tc_fence_after();
-          const uint32_t qoff = (s * 2 * Cfg::kTileBytes) >> 4, dooff = ((s * 2 + 1) * Cfg::kTileBytes) >> 4;
+          const uint32_t qoff = (sq * Cfg::kTileBytes) >> 4, dooff = (sd * Cfg::kTileBytes) >> 4;
           // S^T over P^T of the previous tile (consumed by the dV product
           // issued before); dP^T over dS^T (consumed by dK) and, at d=128,
           // over the previous dQ once it has been loaded out
-          kmajor(kColS, dKd, dRingK + qoff);
+          kmajor(kColS, dKd, dQk + qoff);
           if (Cfg::kDqShared && !(ok = wait_dq_free())) break;
-          kmajor(kColDP, dVd, dRingK + dooff);
+          if (!(ok = mbar_wait(do_full + sd, (q_iter / SD) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
+          tc_fence_after();
+          kmajor(kColDP, dVd, dDok + dooff);
           mma_commit(sd_full);
           if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
           tc_fence_after();
-          accum(kColDV, kColS + kPk, dRingMN + dooff, i > i0);   // dV += P^T dO_i
-          accum(kColDK, kColDP + kPk, dRingMN + qoff, i > i0);   // dK += dS^T Q_i
-          mma_commit(q_empty + s);
+          accum(kColDV, kColS + kPk, dDomn + dooff, i > i0);   // dV += P^T dO_i
+          mma_commit(do_empty + sd);
+          accum(kColDK, kColDP + kPk, dQmn + qoff, i > i0);    // dK += dS^T Q_i
+          mma_commit(q_empty + sq);
           if (!Cfg::kDqShared && !(ok = wait_dq_free())) break;
           // dQ_i = dS K_j: 16 keys (16 rows of 128 bytes in both operands) per product
 #pragma unroll
@@ -311,7 +336,6 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
     __syncwarp();
   }
   } else if (warp < 12) {
-    reg_alloc<kBwdRegsHigh>();
     // ------------------------------------------------------------- key rows
     const int half = (warp - 4) >> 2;          // queries 64*half .. 64*half+63
     const int quarter = warp & 3;
@@ -335,11 +359,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
       const bool key_ok = key < p.N;
       const size_t rbase = static_cast<size_t>(bh) * p.N;
       for (int i = i0; i < n_t; ++i, ++t) {
-        const uint32_t s = t % S;
-        bool w = mbar_wait(q_full + s, (t / S) & 1, p.status, abort_flag, kWhereKvFull, lim);
+        const uint32_t s = t % SQ;
+        bool w = mbar_wait(q_full + s, (t / SQ) & 1, p.status, abort_flag, kWhereKvFull, lim);
         w = w && mbar_wait(sd_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
-        // the dS buffer: free once the previous tile's dQ staging has been read
-        w = w && (t == 0 || mbar_wait(ds_free, (t - 1) & 1, p.status, abort_flag, kWhereDrain, lim));
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
         const float* lse2 = sRows + s * 256;
@@ -418,12 +440,15 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
       }
     }
   } else {
-    reg_alloc<kBwdRegsHigh>();
+    reg_alloc<kBwdRegsDq>();
     // ------------------------------------------------------------ dQ rows
+    // Thread = query row.  The whole dQ tile goes to registers (then the
+    // next dP^T may overwrite the columns), then 32 x 32 fp32 boxes, staged
+    // in this warp's 4 KiB slice of two box buffers, are added into the
+    // accumulator by TMA reduce-add.
     const int quarter = warp & 3;              // rows 32*quarter .. +31 of the Q tile
     const uint32_t tDQ = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColDQ;
-    constexpr int kStageBytes = 16384;                   // one box buffer: 4 warps x 32 rows x 128 bytes
-    uint8_t* stage = sDS + quarter * 4096 + lane * 128;   // this lane's row in box buffer 0
+    uint8_t* stage = sStage + quarter * 4096 + lane * 128;
     const int sw = lane & 7;
     uint32_t t = 0;
     bool ok = true;
@@ -438,46 +463,31 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         bool w = mbar_wait(dq_full, t & 1, p.status, abort_flag, kWhereDrain, lim);
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
-        // 64 columns at a time: load, stage as two 32 x 32 boxes, reduce-add.
-        // dq_empty is signalled once every column has been loaded.
+        uint32_t rr[D];
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tDQ + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(rr + cc * 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(dq_empty);
         const int row0 = i * 128 + quarter * 32;
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
-          uint32_t rr[64];
-          tmem_ld32(tDQ + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(rr));
-          tmem_ld32(tDQ + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
-          tmem_wait_ld();
-          if (hh == D / 64 - 1) {
-            tc_fence_before();
-            mbar_arrive(dq_empty);
-          }
+        for (int m = 0; m < D / 32; ++m) {
+          // buffer m % 2 is free once at most one (the other buffer's) box is still read
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          uint8_t* dst = stage + (m & 1) * Cfg::kStageBytes;
 #pragma unroll
-          for (int mm = 0; mm < 2; ++mm) {
-            const int m = 2 * hh + mm;   // box: columns 32m .. 32m+31, buffer m % 2
-            if (m >= 2) {
-              if (lane == 0) bulk_wait_group_read<1>();   // box m-2 has left this buffer
-              __syncwarp();
-            }
-            uint8_t* dst = stage + mm * kStageBytes;
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-              *reinterpret_cast<uint4*>(dst + ((g ^ sw) << 4)) =
-                  make_uint4(rr[32 * mm + 4 * g], rr[32 * mm + 4 * g + 1], rr[32 * mm + 4 * g + 2],
-                             rr[32 * mm + 4 * g + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (row0 < p.N && 32 * m < p.d_out)
-                tma_reduce_add_3d(&p.tm_dq, sDS + mm * kStageBytes + quarter * 4096, 32 * m, row0, bh);
-              bulk_commit_group();
-            }
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<uint4*>(dst + ((g ^ sw) << 4)) =
+                make_uint4(rr[32 * m + 4 * g], rr[32 * m + 4 * g + 1], rr[32 * m + 4 * g + 2], rr[32 * m + 4 * g + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.N && 32 * m < p.d_out)
+              tma_reduce_add_3d(&p.tm_dq, sStage + (m & 1) * Cfg::kStageBytes + quarter * 4096, 32 * m, row0, bh);
+            bulk_commit_group();
           }
         }
-        if (lane == 0) {
-          bulk_wait_group_read<0>();
-          mbar_arrive(ds_free);
-        }
-        __syncwarp();
       }
     }
     if (lane == 0) bulk_wait_group<0>();

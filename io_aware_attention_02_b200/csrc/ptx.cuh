@@ -271,13 +271,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Four fp32 atomic adds to consecutive global addresses (16-byte aligned),
-// no return value.
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
-               ::"l"(reinterpret_cast<uint64_t>(addr)), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
 // ----------------------------------------------------------------------------
 // Descriptors
 // ----------------------------------------------------------------------------
