@@ -18,11 +18,12 @@
 // Fused kernel, per Q tile i of the unit's key tile j (TMEM columns at d=128:
 // S^T 0-127 | dP^T 128-255 | dV 256-383 | dK 384-511):
 //   MMA   S^T = K Q_i^T, dP^T = V dO_i^T (SS, both K-major)
-//   rows  two warpgroups, thread = key, queries 0-63 and 64-127: P^T and
-//         dS^T, 16-bit, packed into TMEM columns 32-95 of S^T and dP^T (each
-//         warpgroup writes only columns it has already read), and dS into
-//         shared memory (query-contiguous rows, the MN-major A operand of the
-//         dQ product)
+//   rows  two warpgroups, thread = key, queries 0-63 and 64-127.  Phase 1,
+//         as soon as S^T is done: P (fp32) over S^T in place.  Phase 2, once
+//         dP^T is done: P^T and dS^T, 16-bit, packed into TMEM columns 32-95
+//         of S^T and dP^T (each warpgroup writes only columns it has already
+//         read), and dS into shared memory (query-contiguous rows, the
+//         MN-major A operand of the dQ product)
 //   MMA   dV += P^T dO_i, dK += dS^T Q_i (TS), dQ_i = dS K_j (SS, both
 //         MN-major) into the dP^T columns, which dK has just consumed
 //   dQ    one warpgroup, thread = query: TMEM -> registers (the next dP^T
@@ -117,11 +118,14 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
 // The fused kernel
 // ---------------------------------------------------------------------------
 // Register split (setmaxnreg, per warpgroup): 512 threads launch with 128
-// registers each; the TMA/MMA warpgroup gives 32 to the dQ warpgroup, which
-// holds a whole 128-column dQ tile (96 + 128 + 128 + 160 = 4 * 128).
-constexpr int kBwdRegsLow = 96;
-constexpr int kBwdRegsDq = 160;
-static_assert(128 * kBwdRegsLow + 256 * 128 + 128 * kBwdRegsDq <= 512 * 128, "register split exceeds the launch pool");
+// registers each; the TMA/MMA warpgroup gives 40 to the row warpgroups and
+// the dQ warpgroup, which holds a whole 128-column dQ tile
+// (88 + 136 + 136 + 152 = 4 * 128).
+constexpr int kBwdRegsLow = 88;
+constexpr int kBwdRegsRows = 136;
+constexpr int kBwdRegsDq = 152;
+static_assert(128 * kBwdRegsLow + 256 * kBwdRegsRows + 128 * kBwdRegsDq <= 512 * 128,
+              "register split exceeds the launch pool");
 
 template <typename E, int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
@@ -144,17 +148,18 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* sd_full = bars + 2;      // S^T, dP^T in TMEM
+  uint64_t* s_full = bars + 2;       // S^T in TMEM
   uint64_t* p_ready = bars + 3;      // P^T, dS^T in TMEM and dS in shared memory
   uint64_t* dq_full = bars + 4;      // dQ_i in TMEM
   uint64_t* dq_empty = bars + 5;     // dQ_i loaded out of TMEM
   uint64_t* acc_full = bars + 6;     // dV, dK of the unit complete
   uint64_t* drain = bars + 7;
+  uint64_t* dp_full = bars + 8 + 2 * SQ + 2 * SD;   // dP^T in TMEM
   uint64_t* q_full = bars + 8;                 // [SQ] Q tile and its row statistics
   uint64_t* q_empty = bars + 8 + SQ;           // [SQ]
   uint64_t* do_full = bars + 8 + 2 * SQ;       // [SD]
   uint64_t* do_empty = bars + 8 + 2 * SQ + SD; // [SD]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * SQ + 2 * SD);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * SQ + 2 * SD);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
   constexpr int kColDQ = Cfg::kColDQ;
@@ -165,7 +170,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    mbar_init(sd_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     mbar_init(p_ready, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -304,11 +310,12 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           // issued before); dP^T over dS^T (consumed by dK) and, at d=128,
           // over the previous dQ once it has been loaded out
           kmajor(kColS, dKd, dQk + qoff);
+          mma_commit(s_full);
           if (Cfg::kDqShared && !(ok = wait_dq_free())) break;
           if (!(ok = mbar_wait(do_full + sd, (q_iter / SD) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
           tc_fence_after();
           kmajor(kColDP, dVd, dDok + dooff);
-          mma_commit(sd_full);
+          mma_commit(dp_full);
           if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
           tc_fence_after();
           accum(kColDV, kColS + kPk, dDomn + dooff, i > i0);   // dV += P^T dO_i
@@ -336,6 +343,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
     __syncwarp();
   }
   } else if (warp < 12) {
+    if (kBwdRegsRows > 128) reg_alloc<kBwdRegsRows>();
     // ------------------------------------------------------------- key rows
     const int half = (warp - 4) >> 2;          // queries 64*half .. 64*half+63
     const int quarter = warp & 3;
@@ -361,7 +369,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
       for (int i = i0; i < n_t; ++i, ++t) {
         const uint32_t s = t % SQ;
         bool w = mbar_wait(q_full + s, (t / SQ) & 1, p.status, abort_flag, kWhereKvFull, lim);
-        w = w && mbar_wait(sd_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
+        w = w && mbar_wait(s_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
         const float* lse2 = sRows + s * 256;
@@ -369,10 +377,40 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         const int q0 = i * 128;
         // every pair of this tile is visible: no per-element mask
         const bool full = !(CAUSAL && i == j) && q0 + 128 <= p.N && j * 128 + 128 <= p.N;
-        // Chunks of 32 queries, in an order that makes every packed write
-        // land on columns this warpgroup has already read: half 0 reads
-        // 0-63 and writes 32-63 (chunk 1 first), half 1 reads 64-127 and
-        // writes 64-95.
+        // Phase 1 (S^T only, while dP^T may still be computed): P in fp32,
+        // written back over S^T in place.
+#pragma unroll
+        for (int cc0 = 0; cc0 < 2; ++cc0) {
+          const int cc = 2 * half + cc0;
+          uint32_t sr[32];
+          tmem_ld32(tS + cc * 32, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x4 = 0; x4 < 8; ++x4) {
+            const float4 lv = reinterpret_cast<const float4*>(lse2 + cc * 32)[x4];   // broadcast reads
+            const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int x = 4 * x4 + e;
+              float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -l4[e]));
+              if (!full) {
+                const int qg = q0 + cc * 32 + x;
+                const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
+                pr = vis ? pr : 0.f;
+              }
+              sr[x] = __float_as_uint(pr);
+            }
+          }
+          tmem_st32(tS + cc * 32, sr);
+        }
+        tmem_wait_st();
+        w = mbar_wait(dp_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
+        tc_fence_after();
+        // Phase 2: dS = P (dP - D).  Chunks of 32 queries, in an order that
+        // makes every packed write land on columns this warpgroup has
+        // already read: half 0 reads 0-63 and writes 32-63 (chunk 1 first),
+        // half 1 reads 64-127 and writes 64-95.
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
           const int cc = half == 0 ? 1 - n : 2 + n;
@@ -383,26 +421,16 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           uint32_t pp[16], pd[16];
 #pragma unroll
           for (int x4 = 0; x4 < 8; ++x4) {
-            // LSE2 and D of 4 queries (broadcast shared-memory reads)
-            const float4 lv = reinterpret_cast<const float4*>(lse2 + cc * 32)[x4];
             const float4 dv = reinterpret_cast<const float4*>(dvec + cc * 32)[x4];
-            const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
             const float d4[4] = {dv.x, dv.y, dv.z, dv.w};
-            float pv[4], dsv[4];
+            float dsv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int x = 4 * x4 + e;
-              float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -l4[e]));
-              if (!full) {
-                const int qg = q0 + cc * 32 + x;
-                const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
-                pr = vis ? pr : 0.f;
-              }
-              pv[e] = pr;
-              dsv[e] = pr * (__uint_as_float(dr[x]) - d4[e]);
+              dsv[e] = __uint_as_float(sr[x]) * (__uint_as_float(dr[x]) - d4[e]);
             }
-            pp[2 * x4] = pack2<T>(pv[0], pv[1]);
-            pp[2 * x4 + 1] = pack2<T>(pv[2], pv[3]);
+            pp[2 * x4] = pack2<T>(__uint_as_float(sr[4 * x4]), __uint_as_float(sr[4 * x4 + 1]));
+            pp[2 * x4 + 1] = pack2<T>(__uint_as_float(sr[4 * x4 + 2]), __uint_as_float(sr[4 * x4 + 3]));
             pd[2 * x4] = pack2<T>(dsv[0], dsv[1]);
             pd[2 * x4 + 1] = pack2<T>(dsv[2], dsv[3]);
           }
