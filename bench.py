@@ -292,6 +292,24 @@ def run_ours(args, world, rank, local):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     f_nc = flops(B, H, N, d, False)
 
+    if args.only == "bwd":
+        dod = inputs.grad_out(B, H, N, d, seed=rank_seed(rank)).to(dev)
+        binding.fwd(qd, kd, vd, out=o, lse=lse)
+        grads = [torch.empty_like(qd) for _ in range(3)]
+        ws = torch.empty(binding.bwd_workspace_bytes(B, H, N, d, False), dtype=torch.uint8, device=dev)
+
+        def step_b():
+            binding.bwd(qd, kd, vd, o, dod, lse, dq=grads[0], dk=grads[1], dv=grads[2], workspace=ws)
+        ms_b = timed(step_b, args.steps, args.warmup, world) / args.steps
+        code, where = binding.last_status()
+        if code != 0:
+            raise RuntimeError(f"kernel status {code} at {where}")
+        if rank == 0:
+            print(json.dumps({"metric": "attention bwd TFLOP/s (5 products, 10*B*H*N^2*d)",
+                              "value": job_throughput(2.5 * f_nc, world, ms_b), "unit": "TFLOP/s",
+                              "ms_per_step": ms_b, "steps": args.steps, "only": "bwd"}), flush=True)
+        return
+
     def step():
         binding.fwd(qd, kd, vd, causal=False, out=o, lse=lse)
 
@@ -468,8 +486,9 @@ def main():
     ap.add_argument("--ref-total", type=float, default=150.0,
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "main"], default="all",
-                    help="main: time only the bf16 non-causal step (for profiler runs)")
+    ap.add_argument("--only", choices=["all", "main", "bwd"], default="all",
+                    help="main: time only the bf16 non-causal step; bwd: only the fused bf16 "
+                         "non-causal backward of the same workload (for profiler runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="print TFLOP/s for the sequence sweep and the long-context case instead")
     args = ap.parse_args()
