@@ -33,6 +33,8 @@ Modules:
   written out.
 * ``baselines`` -- the per-tensor FP8 and standard FP16 attentions of the
   pages' accuracy experiment.
+* ``decode``    -- fewer queries than keys (decode causal alignment) and the
+  split-KV merge of partial results.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 against closed forms, invariants, a hand-computed two-token example, a
@@ -41,4 +43,4 @@ pure-Python brute force and library routines (``torch`` SDPA in float64,
 print (2.6x, 1.7x) are NOT pinned: "parity unpinned" for those ratios.
 """
 
-from . import attention, backward, baselines, fp8  # noqa: F401
+from . import attention, backward, baselines, decode, fp8  # noqa: F401
