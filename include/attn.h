@@ -233,6 +233,51 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                        int deterministic, int dtype, void* stream);
 
+/*
+ * attn_fwd_splitkv -- 16-bit attention forward for Nq queries against Nk
+ * keys, the keys divided into splits processed in parallel and merged
+ * (the decode-phase parallelisation over the key/value length the pages
+ * attribute to FlashDecoding: "FlashAttention-3" explainer, droidorbit.com,
+ * FAQ "How does FlashAttention-3 compare to FlashDecoding?").  Each split s
+ * computes over its keys J_s the partial result O_s and LSE_s of the
+ * definition above; the merge is the online-softmax rescaling across splits:
+ * LSE = ln sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
+ *   q, o    : [B][H][Nq][d] bf16 or fp16 (per `dtype`); o written.
+ *   k, v    : [B][H][Nk][d] same dtype, read only.
+ *   lse     : [B][H][Nq] fp32 (natural log), written; may be NULL.
+ *   Nq, Nk  : >= 1, B*H*Nq and B*H*Nk < 2^31.
+ *   causal  : 0 or 1.  Query i stands at position Nk - Nq + i: it sees keys
+ *             j <= Nk - Nq + i (requires Nq <= Nk; with Nq = Nk this is
+ *             attn_fwd's mask).
+ *   n_splits: number of key splits per (batch, head, 128-query tile); 0
+ *             picks one from the sizes and the SM count
+ *             (attn_fwd_splitkv_auto_splits); larger than ceil(Nk / 128) is
+ *             clamped to it.  Causal query tiles that see fewer key tiles use
+ *             fewer splits.
+ *   workspace: device memory of at least attn_fwd_splitkv_workspace_bytes(B,
+ *             H, Nq, d, n_splits) bytes (with the split count actually used),
+ *             16-byte aligned, owned by the caller, contents irrelevant:
+ *             fp32 partial O_s [n_splits][B*H][Nq][d] then LSE_s.
+ *   d       : a multiple of 8, at most 128 (64 and 128 natively, others
+ *             zero-padded).
+ *   scale, dtype, stream: as for attn_fwd.
+ * Two kernels on `stream` (splits, then the merge).  Rounding: each split as
+ * attn_fwd (fp32 statistics, P rounded to the input dtype) with O_s kept in
+ * fp32; the merge is fp32; O is rounded once to the input dtype.
+ */
+attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                               int n_splits, int dtype, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Bytes of workspace attn_fwd_splitkv needs for `n_splits` splits (0 for
+ * sizes < 1). */
+size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int d, int n_splits);
+
+/* The split count attn_fwd_splitkv uses when given n_splits = 0, for the
+ * current device (0 for sizes < 1 or a CUDA error). */
+int attn_fwd_splitkv_auto_splits(int B, int H, int Nq, int Nk);
+
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t s);
 

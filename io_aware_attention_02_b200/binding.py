@@ -32,6 +32,9 @@ SIGNATURES = {
     "attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
     "attn_fwd_strided": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _F, _I, _I, _P]),
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_fwd_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P, ctypes.c_size_t, _P]),
+    "attn_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_fwd_splitkv_auto_splits": (_I, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _I, _I,
                       _P]),
 }
@@ -202,6 +205,37 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
                            _stream(q.device))
     _check("attn_bwd", code)
     return dq, dk, dv
+
+
+def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_splits: int = 0,
+                out=None, lse=None, return_lse: bool = True, workspace=None):
+    """O, LSE of q [B, H, Nq, d] against k, v [B, H, Nk, d] through
+    ``attn_fwd_splitkv`` (keys split across CTAs, then merged).  Causal
+    masking aligns the queries with the last Nq key positions."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor [B, H, rows, d]")
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bf16 or all fp16")
+    B, H, Nq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
+        raise ValueError("k and v must be [B, H, Nk, d] matching q")
+    Nk = k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    ns = int(n_splits) if n_splits else int(load().attn_fwd_splitkv_auto_splits(B, H, Nq, Nk))
+    ns = max(1, min(ns, (Nk + 127) // 128))
+    if workspace is None:
+        nbytes = int(load().attn_fwd_splitkv_workspace_bytes(B, H, Nq, d, ns))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
+    code = load().attn_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse) if return_lse else None,
+                                   B, H, Nq, Nk, d, scale, int(bool(causal)), ns, dtype, _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check("attn_fwd_splitkv", code)
+    return o, (lse if return_lse else None)
 
 
 def quant_fp8(x: torch.Tensor, hadamard: bool = False, signs: torch.Tensor | None = None,

@@ -14,6 +14,7 @@
 #include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "quant_fp8.cuh"
+#include "splitkv_sm100.cuh"
 
 namespace {
 
@@ -320,6 +321,53 @@ attn_status_t launch_bwd_fused_c(const attn::BwdParams& p, int sm_count, int cau
                 : launch_bwd_fused<E, D, false>(p, sm_count, o, d_o, s);
 }
 
+// Split-KV forward: split kernel, then the merge.
+template <typename E, int D, bool CAUSAL>
+attn_status_t launch_splitkv(const attn::SplitParams& p, int grid, void* o, float* lse, cudaStream_t stream) {
+  using Cfg = attn::SplitCfg<D>;
+  auto kern = attn::attn_splitkv_kernel<E, D, CAUSAL>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_done = true;
+  }
+  kern<<<grid, Cfg::kThreads, Cfg::kSmem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  const long long warps = static_cast<long long>(p.BH) * p.Nq;
+  attn::attn_splitkv_combine_kernel<E, CAUSAL><<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(
+      p.o_part, p.lse_part, static_cast<E*>(o), lse, p.BH, p.Nq, p.n_kv, p.n_splits, p.q_off, p.d_out);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename E, int D>
+attn_status_t launch_splitkv_c(const attn::SplitParams& p, int grid, int causal, void* o, float* lse,
+                               cudaStream_t s) {
+  return causal ? launch_splitkv<E, D, true>(p, grid, o, lse, s) : launch_splitkv<E, D, false>(p, grid, o, lse, s);
+}
+
+size_t splitkv_workspace_bytes(int B, int H, int Nq, int d, int n_splits) {
+  const size_t rows = static_cast<size_t>(n_splits) * B * H * Nq;
+  return rows * d * sizeof(float) + ((rows * sizeof(float) + 15) / 16) * 16;
+}
+
+// Split count when the caller passes 0: the fewest splits (from enough to
+// cover the SMs) whose work units fill their last round of CTAs to at least
+// 90 %, each split keeping at least two key tiles.
+int splitkv_auto_splits(int BH, int n_qt, int n_kv, int sm_count) {
+  const long long base = static_cast<long long>(BH) * n_qt;
+  const int cap = n_kv / 2 > 1 ? n_kv / 2 : 1;
+  int first = static_cast<int>((sm_count + base - 1) / base);
+  if (first < 1) first = 1;
+  if (first > cap) return cap;
+  for (int n = first; n <= cap && n <= 256; ++n) {
+    const long long units = base * n;
+    const long long rounds = (units + sm_count - 1) / sm_count;
+    if (units * 10 >= rounds * sm_count * 9) return n;
+  }
+  return first;
+}
+
 size_t bwd_rows_bytes(int B, int H, int N) {
   return static_cast<size_t>(B) * H * ((N + 127) / 128) * 256 * sizeof(float);
 }
@@ -619,4 +667,76 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
                : launch_bwd_fused_c<__nv_bfloat16, 128>(p, st->sm_count, causal, o, d_o, s);
   return d64 ? launch_bwd_fused_c<__half, 64>(p, st->sm_count, causal, o, d_o, s)
              : launch_bwd_fused_c<__half, 128>(p, st->sm_count, causal, o, d_o, s);
+}
+
+extern "C" size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int d, int n_splits) {
+  if (B < 1 || H < 1 || Nq < 1 || d < 1 || n_splits < 1) return 0;
+  return splitkv_workspace_bytes(B, H, Nq, d, n_splits);
+}
+
+extern "C" int attn_fwd_splitkv_auto_splits(int B, int H, int Nq, int Nk) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return 0;
+  DeviceState* st = nullptr;
+  if (device_state(&st) != ATTN_OK) return 0;
+  return splitkv_auto_splits(B * H, (Nq + 127) / 128, (Nk + 127) / 128, st->sm_count);
+}
+
+extern "C" attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                                          int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                                          int n_splits, int dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || workspace == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * Nk >= (1ll << 31) || static_cast<long long>(B) * H * Nq >= (1ll << 31))
+    return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq > Nk) return ATTN_ERR_INVALID_ARG;   // every query must see at least one key
+  if (n_splits < 0) return ATTN_ERR_INVALID_ARG;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d > 128 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  const void* p16[] = {q, k, v, o, workspace};
+  for (const void* x : p16)
+    if (!aligned16(x)) return ATTN_ERR_MISALIGNED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  attn_status_t r;
+  DeviceState* st = nullptr;
+  if ((r = device_state(&st)) != ATTN_OK) return r;
+  const int BH = B * H;
+  const int n_qt = (Nq + 127) / 128, n_kv = (Nk + 127) / 128;
+  if (n_splits == 0) n_splits = splitkv_auto_splits(BH, n_qt, n_kv, st->sm_count);
+  if (n_splits > n_kv) n_splits = n_kv;
+  if (static_cast<long long>(BH) * n_qt * n_splits >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < splitkv_workspace_bytes(B, H, Nq, d, n_splits)) return ATTN_ERR_INVALID_ARG;
+  const CUtensorMapDataType dt =
+      dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  attn::SplitParams p{};
+  if ((r = make_map(&p.tm_q, q, dt, 2, B, H, Nq, d, contiguous(H, Nq, d), 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k, dt, 2, B, H, Nk, d, contiguous(H, Nk, d), 64)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v, dt, 2, B, H, Nk, d, contiguous(H, Nk, d), 64)) != ATTN_OK) return r;
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = p.o_part + static_cast<size_t>(n_splits) * BH * Nq * d;
+  p.status = st->status;
+  p.BH = BH;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.n_qt = n_qt;
+  p.n_kv = n_kv;
+  p.n_splits = n_splits;
+  p.n_units = BH * n_qt * n_splits;
+  p.q_off = Nk - Nq;
+  p.d_out = d;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = wait_limit_ns();
+  const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool d64 = d <= 64;
+  if (dtype == ATTN_BF16)
+    return d64 ? launch_splitkv_c<__nv_bfloat16, 64>(p, grid, causal, o, lse, s)
+               : launch_splitkv_c<__nv_bfloat16, 128>(p, grid, causal, o, lse, s);
+  return d64 ? launch_splitkv_c<__half, 64>(p, grid, causal, o, lse, s)
+             : launch_splitkv_c<__half, 128>(p, grid, causal, o, lse, s);
 }

@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
     assert _declared() == sorted(["attn_fwd", "attn_quant_fp8", "attn_fwd_fp8", "attn_last_status",
                                   "attn_status_string", "attn_debug_set_fault",
                                   "attn_fwd_noalloc", "attn_fwd_strided", "attn_bwd",
-                                  "attn_bwd_workspace_bytes"])
+                                  "attn_bwd_workspace_bytes", "attn_fwd_splitkv",
+                                  "attn_fwd_splitkv_workspace_bytes", "attn_fwd_splitkv_auto_splits"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -143,6 +144,39 @@ def test_bwd_validation(lib, det):
     assert call(dtype=2) == binding.ATTN_ERR_UNSUPPORTED
     assert call(dk=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
     assert call(ws=GOOD + 4) == binding.ATTN_ERR_MISALIGNED
+    assert call(lse=GOOD + 2) == binding.ATTN_ERR_MISALIGNED
+
+
+def test_splitkv_workspace_size(lib):
+    # fp32 partial O (n_splits x B*H x Nq x d) then LSE (padded to 16 bytes)
+    assert lib.attn_fwd_splitkv_workspace_bytes(2, 3, 5, 64, 4) == 4 * 6 * 5 * 64 * 4 + 4 * 6 * 5 * 4
+    assert lib.attn_fwd_splitkv_workspace_bytes(1, 1, 1, 8, 3) == 3 * 8 * 4 + 16
+    assert lib.attn_fwd_splitkv_workspace_bytes(1, 1, 0, 8, 3) == 0
+    assert lib.attn_fwd_splitkv_workspace_bytes(1, 1, 4, 8, 0) == 0
+
+
+def test_splitkv_validation(lib):
+    F = lib.attn_fwd_splitkv
+    ws = lib.attn_fwd_splitkv_workspace_bytes(1, 2, 4, 64, 3)
+
+    def call(**kw):
+        a = dict(q=GOOD, k=GOOD, v=GOOD, o=GOOD, lse=None, B=1, H=2, Nq=4, Nk=1000, d=64, scale=0.125,
+                 causal=0, ns=3, dtype=0, ws=GOOD, ws_bytes=ws)
+        a.update(kw)
+        return F(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["scale"],
+                 a["causal"], a["ns"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+    assert call(q=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(ws=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(Nq=0) == binding.ATTN_ERR_INVALID_ARG
+    assert call(Nk=0) == binding.ATTN_ERR_INVALID_ARG
+    assert call(causal=1, Nq=2000) == binding.ATTN_ERR_INVALID_ARG     # queries past the keys
+    assert call(ns=-1) == binding.ATTN_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == binding.ATTN_ERR_INVALID_ARG
+    assert call(d=136) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(d=100) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(dtype=5) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(o=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
     assert call(lse=GOOD + 2) == binding.ATTN_ERR_MISALIGNED
 
 
