@@ -355,6 +355,28 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"backward kernel status {code} at {where}")
     del dq, dk, dv, dod
 
+    # decode shape through the split-KV path: one query per (b, h) against a
+    # 32K-token KV cache; HBM-bound (K and V read once)
+    DB, DH, DNk = 8, 32, 32768
+    qdec = torch.randn(DB, DH, 1, d, device=dev, dtype=torch.bfloat16)
+    kdec = torch.randn(DB, DH, DNk, d, device=dev, dtype=torch.bfloat16)
+    vdec = torch.randn_like(kdec)
+    odec = torch.empty_like(qdec)
+    ldec = torch.empty((DB, DH, 1), dtype=torch.float32, device=dev)
+    nsd = int(binding.lib().attn_fwd_splitkv_auto_splits(DB, DH, 1, DNk))
+    wsd = torch.empty(int(binding.lib().attn_fwd_splitkv_workspace_bytes(DB, DH, 1, d, nsd)), dtype=torch.uint8,
+                      device=dev)
+
+    def step_dec():
+        binding.fwd_splitkv(qdec, kdec, vdec, causal=True, n_splits=nsd, out=odec, lse=ldec, workspace=wsd)
+    nd = max(3, args.steps // 4)
+    ms_dec = timed(step_dec, nd, args.warmup, world) / nd
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"split-KV kernel status {code} at {where}")
+    kv_bytes_dec = 2 * DB * DH * DNk * d * 2
+    del qdec, kdec, vdec, odec, ldec, wsd
+
     # FP8 variant: outlier inputs, Hadamard rotation of Q and K, 128 x d block scales
     qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank_seed(rank), outliers=True))
     signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
@@ -430,6 +452,11 @@ def run_ours(args, world, rank, local):
             "bf16_backward_noncausal_deterministic": {
                 "tflops": 2.5 * f_nc / (bwd_ms[(False, True)] * 1e-3) / 1e12, "ms": bwd_ms[(False, True)],
                 "kernels_per_call": 2, "path": "dQ kernel then dK/dV kernel, no atomics"},
+            "bf16_decode_splitkv": {
+                "shape": f"B={DB},H={DH},Nq=1,Nk={DNk},d={d} causal (inputs torch.randn)",
+                "splits": nsd, "ms": ms_dec, "kv_read_GBs": kv_bytes_dec / (ms_dec * 1e-3) / 1e9,
+                "frac_of_measured_hbm": kv_bytes_dec / (ms_dec * 1e-3) / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
+                "kernels_per_call": 2},
             "fp8_e4m3_hadamard_noncausal": {
                 "tflops": tf_8, "ms": ms_8, "pct_of_spec_fp8_peak": 100 * tf_8 / SPEC_FP8_TFLOPS,
                 "quant_ms_qkv": ms_q,
