@@ -502,6 +502,39 @@ def run_sweep(args):
         raise RuntimeError(f"kernel status {code} at {where}")
 
 
+def run_ablation(args):
+    """The pages' ablation shape {B=4, N=8448, H=16, d=128}, non-causal, bf16:
+    attn_fwd (two query tiles per CTA in ping-pong, S over P in TMEM) against
+    the same attention through attn_fwd_splitkv with one split (one query
+    tile per CTA, S double-buffered in TMEM, no ping-pong between tiles).
+    Runs alternate A/B/A/B in one process; one JSON line with the medians."""
+    from io_aware_attention_02_b200 import binding
+    torch.cuda.set_device(0)
+    B, H, N, d = 4, 16, 8448, 128
+    g = torch.Generator(device="cuda").manual_seed(0)
+    q, k, v = (torch.randn(B, H, N, d, device="cuda", dtype=torch.bfloat16, generator=g) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty(int(binding.lib().attn_fwd_splitkv_workspace_bytes(B, H, N, d, 1)), dtype=torch.uint8,
+                     device="cuda")
+    arms = {"pingpong_two_tiles": lambda: binding.fwd(q, k, v, out=o, lse=lse),
+            "one_tile_s_double_buffered": lambda: binding.fwd_splitkv(q, k, v, n_splits=1, out=o, lse=lse,
+                                                                      workspace=ws)}
+    res = {name: [] for name in arms}
+    steps = max(5, args.steps // 20)
+    for _ in range(4):
+        for name, fn in arms.items():
+            res[name].append(timed(fn, steps, 3, 1) / steps)
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} at {where}")
+    f = flops(B, H, N, d, False)
+    print(json.dumps({"ablation": True, "B": B, "H": H, "N": N, "d": d, "causal": False,
+                      **{name: {"ms": statistics.median(v), "tflops": f / (statistics.median(v) * 1e-3) / 1e12}
+                         for name, v in res.items()},
+                      "data": "torch.randn bf16 (timing only)"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -518,9 +551,14 @@ def main():
                          "non-causal backward of the same workload (for profiler runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="print TFLOP/s for the sequence sweep and the long-context case instead")
+    ap.add_argument("--ablation", action="store_true",
+                    help="print the ping-pong ablation at the pages' {4, 8448, 16, 128} shape instead")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.ablation:
+        run_ablation(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
