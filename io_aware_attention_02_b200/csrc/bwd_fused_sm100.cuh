@@ -19,11 +19,12 @@
 // S^T 0-127 | dP^T 128-255 | dV 256-383 | dK 384-511):
 //   MMA   S^T = K Q_i^T, dP^T = V dO_i^T (SS, both K-major)
 //   rows  two warpgroups, thread = key, queries 0-63 and 64-127.  Phase 1,
-//         as soon as S^T is done: P (fp32) over S^T in place.  Phase 2, once
-//         dP^T is done: P^T and dS^T, 16-bit, packed into TMEM columns 32-95
-//         of S^T and dP^T (each warpgroup writes only columns it has already
-//         read), and dS into shared memory (query-contiguous rows, the
-//         MN-major A operand of the dQ product)
+//         as soon as S^T is done: P^T, 16-bit, packed into TMEM columns 32-95
+//         of S^T (each warpgroup writes only columns it has already read);
+//         dV += P^T dO_i starts then and releases dO_i.  Phase 2, once dP^T
+//         is done: dS = P (dP - D) from that 16-bit P, packed into columns
+//         32-95 of dP^T, and dS into shared memory (query-contiguous rows,
+//         the MN-major A operand of the dQ product)
 //   MMA   dV += P^T dO_i, dK += dS^T Q_i (TS), dQ_i = dS K_j (SS, both
 //         MN-major) into the dP^T columns, which dK has just consumed
 //   dQ    one warpgroup, thread = query: TMEM -> registers (the next dP^T
@@ -154,12 +155,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   uint64_t* dq_empty = bars + 5;     // dQ_i loaded out of TMEM
   uint64_t* acc_full = bars + 6;     // dV, dK of the unit complete
   uint64_t* drain = bars + 7;
-  uint64_t* dp_full = bars + 8 + 2 * SQ + 2 * SD;   // dP^T in TMEM
   uint64_t* q_full = bars + 8;                 // [SQ] Q tile and its row statistics
   uint64_t* q_empty = bars + 8 + SQ;           // [SQ]
   uint64_t* do_full = bars + 8 + 2 * SQ;       // [SD]
   uint64_t* do_empty = bars + 8 + 2 * SQ + SD; // [SD]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * SQ + 2 * SD);
+  uint64_t* dp_full = bars + 8 + 2 * SQ + 2 * SD;   // dP^T in TMEM
+  uint64_t* pt_ready = bars + 9 + 2 * SQ + 2 * SD;  // packed P^T in TMEM (both row warpgroups)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 2 * SQ + 2 * SD);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
   constexpr int kColDQ = Cfg::kColDQ;
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
     mbar_init(kv_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
+    mbar_init(pt_ready, 256);
     mbar_init(p_ready, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -316,10 +319,14 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           tc_fence_after();
           kmajor(kColDP, dVd, dDok + dooff);
           mma_commit(dp_full);
-          if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
+          // dV as soon as P^T is packed (phase 1): dO is released while the
+          // row warpgroups still compute dS
+          if (!(ok = mbar_wait(pt_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
           tc_fence_after();
           accum(kColDV, kColS + kPk, dDomn + dooff, i > i0);   // dV += P^T dO_i
           mma_commit(do_empty + sd);
+          if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
+          tc_fence_after();
           accum(kColDK, kColDP + kPk, dQmn + qoff, i > i0);    // dK += dS^T Q_i
           mma_commit(q_empty + sq);
           if (!Cfg::kDqShared && !(ok = wait_dq_free())) break;
@@ -377,64 +384,66 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         const int q0 = i * 128;
         // every pair of this tile is visible: no per-element mask
         const bool full = !(CAUSAL && i == j) && q0 + 128 <= p.N && j * 128 + 128 <= p.N;
-        // Phase 1 (S^T only, while dP^T may still be computed): P in fp32,
-        // written back over S^T in place.
-#pragma unroll
-        for (int cc0 = 0; cc0 < 2; ++cc0) {
-          const int cc = 2 * half + cc0;
-          uint32_t sr[32];
-          tmem_ld32(tS + cc * 32, sr);
+        // Phase 1 (S^T only, while dP^T may still be computed): P for this
+        // warpgroup's 64 queries, packed to 16 bits into columns
+        // 32 + 32*half .. of S^T (inside the 64 columns it has just read) --
+        // the A operand of dV, which starts as soon as both halves are in.
+        {
+          uint32_t sr[64];
+          tmem_ld32(tS + (2 * half) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr));
+          tmem_ld32(tS + (2 * half + 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
           tmem_wait_ld();
+          uint32_t pp[32];
 #pragma unroll
-          for (int x4 = 0; x4 < 8; ++x4) {
-            const float4 lv = reinterpret_cast<const float4*>(lse2 + cc * 32)[x4];   // broadcast reads
+          for (int x4 = 0; x4 < 16; ++x4) {
+            const float4 lv = reinterpret_cast<const float4*>(lse2 + half * 64)[x4];   // broadcast reads
             const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+            float pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int x = 4 * x4 + e;
               float pr = ex2_approx(fmaf(__uint_as_float(sr[x]), c2, -l4[e]));
               if (!full) {
-                const int qg = q0 + cc * 32 + x;
+                const int qg = q0 + half * 64 + x;
                 const bool vis = key_ok && qg < p.N && (!CAUSAL || key <= qg);
                 pr = vis ? pr : 0.f;
               }
-              sr[x] = __float_as_uint(pr);
+              pv[e] = pr;
             }
+            pp[2 * x4] = pack2<T>(pv[0], pv[1]);
+            pp[2 * x4 + 1] = pack2<T>(pv[2], pv[3]);
           }
-          tmem_st32(tS + cc * 32, sr);
+          tmem_st32(tS + kPk + half * 32, pp);
         }
         tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(pt_ready);
         w = mbar_wait(dp_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
-        // Phase 2: dS = P (dP - D).  Chunks of 32 queries, in an order that
-        // makes every packed write land on columns this warpgroup has
-        // already read: half 0 reads 0-63 and writes 32-63 (chunk 1 first),
-        // half 1 reads 64-127 and writes 64-95.
+        // Phase 2: dS = P (dP - D) with the 16-bit P of phase 1.  Chunks of 32
+        // queries, in an order that makes every packed dS^T write land on
+        // columns of dP^T this warpgroup has already read: half 0 reads 0-63
+        // and writes 32-63 (chunk 1 first), half 1 reads 64-127 and writes
+        // 64-95.
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
           const int cc = half == 0 ? 1 - n : 2 + n;
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tS + cc * 32, sr);
+          uint32_t pr16[16], dr[32];
+          tmem_ld16(tS + kPk + cc * 16, pr16);
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
-          uint32_t pp[16], pd[16];
+          uint32_t pd[16];
 #pragma unroll
           for (int x4 = 0; x4 < 8; ++x4) {
             const float4 dv = reinterpret_cast<const float4*>(dvec + cc * 32)[x4];
-            const float d4[4] = {dv.x, dv.y, dv.z, dv.w};
-            float dsv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int x = 4 * x4 + e;
-              dsv[e] = __uint_as_float(sr[x]) * (__uint_as_float(dr[x]) - d4[e]);
-            }
-            pp[2 * x4] = pack2<T>(__uint_as_float(sr[4 * x4]), __uint_as_float(sr[4 * x4 + 1]));
-            pp[2 * x4 + 1] = pack2<T>(__uint_as_float(sr[4 * x4 + 2]), __uint_as_float(sr[4 * x4 + 3]));
-            pd[2 * x4] = pack2<T>(dsv[0], dsv[1]);
-            pd[2 * x4 + 1] = pack2<T>(dsv[2], dsv[3]);
+            const float2 p01 = unpack2<T>(pr16[2 * x4]);
+            const float2 p23 = unpack2<T>(pr16[2 * x4 + 1]);
+            pd[2 * x4] = pack2<T>(p01.x * (__uint_as_float(dr[4 * x4]) - dv.x),
+                                  p01.y * (__uint_as_float(dr[4 * x4 + 1]) - dv.y));
+            pd[2 * x4 + 1] = pack2<T>(p23.x * (__uint_as_float(dr[4 * x4 + 2]) - dv.z),
+                                      p23.y * (__uint_as_float(dr[4 * x4 + 3]) - dv.w));
           }
-          tmem_st16(tS + kPk + cc * 16, pp);
           tmem_st16(tDP + kPk + cc * 16, pd);
           // dS row `key`, queries 32cc..32cc+31: 16-byte groups 4(cc%2)..+3 of
           // this half's chunk, 128-byte swizzled
