@@ -292,6 +292,28 @@ def run_ours(args, world, rank, local):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     f_nc = flops(B, H, N, d, False)
 
+    if args.only == "decode":
+        DB, DH, DNk = 8, 32, 32768
+        qdec = torch.randn(DB, DH, 1, d, device=dev, dtype=torch.bfloat16)
+        kdec = torch.randn(DB, DH, DNk, d, device=dev, dtype=torch.bfloat16)
+        vdec = torch.randn_like(kdec)
+        odec = torch.empty_like(qdec)
+        ldec = torch.empty((DB, DH, 1), dtype=torch.float32, device=dev)
+        nsd = int(binding.lib().attn_fwd_splitkv_auto_splits(DB, DH, 1, DNk))
+        wsd = torch.empty(int(binding.lib().attn_fwd_splitkv_workspace_bytes(DB, DH, 1, d, nsd)),
+                          dtype=torch.uint8, device=dev)
+        ms_dec = timed(lambda: binding.fwd_splitkv(qdec, kdec, vdec, causal=True, n_splits=nsd, out=odec,
+                                                   lse=ldec, workspace=wsd), args.steps, args.warmup, world) / args.steps
+        code, where = binding.last_status()
+        if code != 0:
+            raise RuntimeError(f"kernel status {code} at {where}")
+        if rank == 0:
+            print(json.dumps({"metric": "split-KV decode K/V read GB/s", "unit": "GB/s",
+                              "value": world * 2 * DB * DH * DNk * d * 2 / (ms_dec * 1e-3) / 1e9,
+                              "ms_per_step": ms_dec, "splits": nsd, "steps": args.steps, "only": "decode"}),
+                  flush=True)
+        return
+
     if args.only == "bwd":
         dod = inputs.grad_out(B, H, N, d, seed=rank_seed(rank)).to(dev)
         binding.fwd(qd, kd, vd, out=o, lse=lse)
@@ -546,9 +568,10 @@ def main():
     ap.add_argument("--ref-total", type=float, default=150.0,
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "main", "bwd"], default="all",
+    ap.add_argument("--only", choices=["all", "main", "bwd", "decode"], default="all",
                     help="main: time only the bf16 non-causal step; bwd: only the fused bf16 "
-                         "non-causal backward of the same workload (for profiler runs)")
+                         "non-causal backward of the same workload; decode: only the split-KV decode "
+                         "variant (for profiler runs)")
     ap.add_argument("--sweep", action="store_true",
                     help="print TFLOP/s for the sequence sweep and the long-context case instead")
     ap.add_argument("--ablation", action="store_true",
