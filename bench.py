@@ -293,7 +293,7 @@ def run_ours(args, world, rank, local):
     f_nc = flops(B, H, N, d, False)
 
     if args.only == "decode":
-        DB, DH, DNk = 8, 32, 32768
+        DB, DH, DNk = 8, 32, args.decode_nk
         qdec = torch.randn(DB, DH, 1, d, device=dev, dtype=torch.bfloat16)
         kdec = torch.randn(DB, DH, DNk, d, device=dev, dtype=torch.bfloat16)
         vdec = torch.randn_like(kdec)
@@ -572,6 +572,8 @@ def main():
                     help="main: time only the bf16 non-causal step; bwd: only the fused bf16 "
                          "non-causal backward of the same workload; decode: only the split-KV decode "
                          "variant (for profiler runs)")
+    ap.add_argument("--decode-nk", type=int, default=32768,
+                    help="KV length of the --only decode run (smaller for profiler captures)")
     ap.add_argument("--sweep", action="store_true",
                     help="print TFLOP/s for the sequence sweep and the long-context case instead")
     ap.add_argument("--ablation", action="store_true",
