@@ -201,29 +201,38 @@ def timed(fn, steps, warmup, world):
 # CPU oracle baseline (rank 0, one GPU only)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(q, k, v, causal, budget_s=15.0, gpu_out=None):
-    """Time the fp64 oracle on sampled query rows of a few heads.
+def oracle_sample(q, k, v, causal, budget_s=15.0, gpu_out=None, single_thread=True):
+    """Time the fp64 oracle on a bounded sample of the workload.
 
-    Rows per head are chosen so that the work takes roughly `budget_s`.
-    Returns the cpu_baseline dict (value in TFLOP/s, same convention as the
-    GPU figure, counted on the rows computed).
+    Whole heads (every query row) while the budget allows more than four of
+    them, else sampled rows of four heads; sized so the work takes roughly
+    `budget_s`.  With `single_thread`, also times 64 rows on one thread.  Returns the cpu_baseline
+    dict (value in TFLOP/s, same convention as the GPU figure, counted on the
+    rows computed).
     """
     from oracle import attention as A
     try:
-        from threadpoolctl import threadpool_info
+        from threadpoolctl import threadpool_info, threadpool_limits
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
+        threadpool_limits = None
         cores = len(os.sched_getaffinity(0))
     B, H, N, d = q.shape
     scale = 1.0 / math.sqrt(d)
-    heads = [(0, 0), (B - 1, H - 1), (B // 2, H // 2), (1 % B, 3 % H)]
-    # calibrate on 64 rows of one head
-    rows = inputs.sample_rows(N, 64, seed=11)
+    # calibrate (after one warm call) on 256 rows of one head
+    rows = inputs.sample_rows(N, 256, seed=11)
+    A.attention_head(q[0, 0], k[0, 0], v[0, 0], scale, causal, rows[:16])
     t0 = time.perf_counter()
     A.attention_head(q[0, 0], k[0, 0], v[0, 0], scale, causal, rows)
     per_row = (time.perf_counter() - t0) / len(rows)
-    n_rows = int(max(64, min(N, budget_s / max(per_row, 1e-9) / len(heads))))
-    rows = inputs.sample_rows(N, n_rows, seed=12)
+    per_head = per_row * N
+    if 4 * per_head <= budget_s:
+        n_heads = int(min(B * H, max(4, budget_s // per_head)))
+        rows = np.arange(N, dtype=np.int64)
+    else:
+        n_heads = 4
+        rows = inputs.sample_rows(N, int(max(64, min(N, budget_s / per_row / 4))), seed=12)
+    heads = [(i % B, (i * 5 + i // B) % H) for i in range(n_heads)]
     errs = []
     t0 = time.perf_counter()
     for b, h in heads:
@@ -240,6 +249,14 @@ def oracle_sample(q, k, v, causal, budget_s=15.0, gpu_out=None):
            "sample": f"{len(rows)} query rows x {len(heads)} heads of B={B},H={H},N={N},d={d} "
                      f"{'causal' if causal else 'non-causal'} (numpy fp64, full keys)",
            "seconds": dt}
+    if single_thread and threadpool_limits is not None:
+        rows1 = inputs.sample_rows(N, 64, seed=13)
+        with threadpool_limits(limits=1):
+            t1 = time.perf_counter()
+            A.attention_head(q[0, 0], k[0, 0], v[0, 0], scale, causal, rows1)
+            dt1 = time.perf_counter() - t1
+        out["single_thread"] = {"value": len(rows1) * 4.0 * N * d / (2 if causal else 1) / dt1 / 1e12,
+                                "unit": "TFLOP/s", "sample": f"{len(rows1)} rows of one head"}
     if errs:
         e = np.array(errs)
         out["parity_sample"] = {"max_abs_dO": float(e[:, 0].max()),
@@ -263,9 +280,9 @@ def run_reference(args, world, rank):
     # about --ref-total seconds of CPU work
     budget = max(0.05, min(args.ref_budget, args.ref_total / (args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(q, k, v, False, budget_s=budget)
+        oracle_sample(q, k, v, False, budget_s=budget, single_thread=False)
     for _ in range(args.steps):
-        cb = oracle_sample(q, k, v, False, budget_s=budget)
+        cb = oracle_sample(q, k, v, False, budget_s=budget, single_thread=False)
         per_step.append(cb["seconds"])
     val = cb["value"]
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 1,
