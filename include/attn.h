@@ -278,6 +278,36 @@ size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int d, int n_split
  * current device (0 for sizes < 1 or a CUDA error). */
 int attn_fwd_splitkv_auto_splits(int B, int H, int Nq, int Nk);
 
+/*
+ * attn_fwd_host -- attn_fwd on HOST buffers, the transfers overlapped with
+ * the computation: the B*H heads are processed in chunks (about an eighth
+ * of the heads each) through two device slots in `workspace`; the
+ * host-to-device copies of chunk c+1 (one internal stream) and the
+ * device-to-host copies of chunk c-1 (another) run while chunk c computes on
+ * `stream`.  One cudaMemcpyAsync per tensor and chunk.
+ *   q_host, k_host, v_host : [B][H][N][d] bf16 / fp16 in host memory (pinned
+ *             memory for the copies to overlap; pageable memory works but
+ *             its copies do not overlap).
+ *   o_host  : [B][H][N][d] same dtype, host memory, written.
+ *   lse_host: [B][H][N] fp32 host memory, written; may be NULL.
+ *   workspace: device memory of at least attn_fwd_host_workspace_bytes(B, H,
+ *             N, d) bytes, 16-byte aligned, owned by the caller.
+ *   B, H, N, d, scale, causal, dtype: as for attn_fwd.
+ * Asynchronous like attn_fwd: the call returns once everything is enqueued;
+ * the results are in host memory when `stream` has completed (synchronize
+ * it before reading o_host / lse_host).  The copies start after the work
+ * already queued on `stream`.  The library keeps two internal streams and
+ * six events per device (created on first use); concurrent calls on one
+ * device from several host threads are not supported.  Outputs are
+ * bit-identical to attn_fwd on the same inputs.
+ */
+attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                            float* lse_host, int B, int H, int N, int d, float scale, int causal, int dtype,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace attn_fwd_host needs (0 for sizes < 1). */
+size_t attn_fwd_host_workspace_bytes(int B, int H, int N, int d);
+
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t s);
 

@@ -35,6 +35,8 @@ SIGNATURES = {
     "attn_fwd_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P, ctypes.c_size_t, _P]),
     "attn_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv_auto_splits": (_I, [_I, _I, _I, _I]),
+    "attn_fwd_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P, ctypes.c_size_t, _P]),
+    "attn_fwd_host_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _I, _I,
                       _P]),
 }
@@ -235,6 +237,41 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_spl
                                    B, H, Nq, Nk, d, scale, int(bool(causal)), ns, dtype, _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(q.device))
     _check("attn_fwd_splitkv", code)
+    return o, (lse if return_lse else None)
+
+
+def fwd_host(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+             return_lse: bool = True, workspace=None, device=None):
+    """O, LSE of host (CPU) tensors [B, H, N, d] through ``attn_fwd_host``:
+    the copies to and from the GPU overlap the computation, chunk by chunk.
+
+    Inputs should be pinned (``tensor.pin_memory()``) for the overlap; the
+    outputs are allocated pinned when not given.  The call is asynchronous on
+    the current stream of ``device`` (default: the current device):
+    synchronize before reading the results.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor [B, H, N, d]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must all be bf16 or all fp16")
+    B, H, N, d = q.shape
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty(q.shape, dtype=q.dtype).pin_memory() if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    if workspace is None:
+        nbytes = int(load().attn_fwd_host_workspace_bytes(B, H, N, d))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    dtype = ATTN_BF16 if q.dtype == torch.bfloat16 else ATTN_FP16
+    with torch.cuda.device(dev):
+        code = load().attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse) if return_lse else None,
+                                    B, H, N, d, scale, int(bool(causal)), dtype, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("attn_fwd_host", code)
     return o, (lse if return_lse else None)
 
 

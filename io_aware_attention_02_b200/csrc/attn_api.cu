@@ -740,3 +740,130 @@ extern "C" attn_status_t attn_fwd_splitkv(const void* q, const void* k, const vo
   return d64 ? launch_splitkv_c<__half, 64>(p, grid, causal, o, lse, s)
              : launch_splitkv_c<__half, 128>(p, grid, causal, o, lse, s);
 }
+
+// ---------------------------------------------------------------------------
+// Host-buffer forward with transfers overlapped with compute (see
+// include/attn.h).  Heads are processed in chunks through two device slots:
+// H2D copies of chunk c+1 on one internal stream and D2H copies of chunk c-1
+// on another run while chunk c computes on the caller's stream.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr, in_done[2] = {nullptr, nullptr}, comp_done[2] = {nullptr, nullptr},
+              out_done[2] = {nullptr, nullptr};
+};
+HostPipe g_pipe[kMaxDevices];
+
+attn_status_t host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return ATTN_OK;
+}
+
+// Heads per chunk: about an eighth of the heads (at least one).  The first
+// chunk's copy-in and the last chunk's compute and copy-out are not
+// overlapped, so smaller chunks shorten that fill and drain.
+int host_chunk_heads(int BH) { return BH >= 8 ? (BH + 7) / 8 : 1; }
+
+size_t host_slot_bytes(int chunk, int N, int d) {
+  const size_t t = static_cast<size_t>(chunk) * N * d * 2;   // one 16-bit [chunk][N][d] tensor
+  const size_t l = ((static_cast<size_t>(chunk) * N * 4 + 255) / 256) * 256;
+  return ((4 * t + 255) / 256) * 256 + l;                    // q, k, v, o, then lse
+}
+
+}  // namespace
+
+extern "C" size_t attn_fwd_host_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  return 2 * host_slot_bytes(host_chunk_heads(B * H), N, d);
+}
+
+extern "C" attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                       float* lse_host, int B, int H, int N, int d, float scale, int causal,
+                                       int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || o_host == nullptr || workspace == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  attn_status_t r = common_checks(B, H, N, scale, causal);
+  if (r != ATTN_OK) return r;
+  if (d < 1) return ATTN_ERR_INVALID_ARG;
+  if (d > 256 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  const int BH = B * H;
+  const int chunk = host_chunk_heads(BH);
+  const size_t slot = host_slot_bytes(chunk, N, d);
+  if (workspace_bytes < 2 * slot) return ATTN_ERR_INVALID_ARG;
+  HostPipe* hp = nullptr;
+  if ((r = host_pipe(&hp)) != ATTN_OK) return r;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t row_bytes = static_cast<size_t>(N) * d * 2;    // one head of one tensor
+  const size_t t_bytes = static_cast<size_t>(chunk) * row_bytes;
+  const size_t t_pad = ((4 * t_bytes + 255) / 256) * 256;
+  // copies of this call start after the work already queued on `stream`
+  if (cudaEventRecord(hp->start, s) != cudaSuccess || cudaStreamWaitEvent(hp->s_in, hp->start, 0) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int n_chunks = (BH + chunk - 1) / chunk;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int i = c & 1;
+    const int h0 = c * chunk;
+    const int nh = BH - h0 < chunk ? BH - h0 : chunk;
+    char* base = static_cast<char*>(workspace) + i * slot;
+    char* dq = base;
+    char* dk = base + t_bytes;
+    char* dv = base + 2 * t_bytes;
+    char* dout = base + 3 * t_bytes;
+    float* dlse = reinterpret_cast<float*>(base + t_pad);
+    const size_t off = static_cast<size_t>(h0) * row_bytes;
+    const size_t bytes = static_cast<size_t>(nh) * row_bytes;
+    // the slot is free once its previous results have been copied out (the
+    // wait is a no-op for an event never recorded)
+    if (cudaStreamWaitEvent(hp->s_in, hp->out_done[i], 0) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyAsync(dq, static_cast<const char*>(q_host) + off, bytes, cudaMemcpyHostToDevice, hp->s_in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(dk, static_cast<const char*>(k_host) + off, bytes, cudaMemcpyHostToDevice, hp->s_in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(dv, static_cast<const char*>(v_host) + off, bytes, cudaMemcpyHostToDevice, hp->s_in) !=
+            cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaEventRecord(hp->in_done[i], hp->s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(s, hp->in_done[i], 0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    const Strides cs = contiguous(nh, N, d);
+    if ((r = fwd16(dq, dk, dv, dout, lse_host ? dlse : nullptr, 1, nh, N, d, cs, cs, cs, cs, scale, causal, dtype,
+                   stream)) != ATTN_OK)
+      return r;
+    if (cudaEventRecord(hp->comp_done[i], s) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->s_out, hp->comp_done[i], 0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaMemcpyAsync(static_cast<char*>(o_host) + off, dout, bytes, cudaMemcpyDeviceToHost, hp->s_out) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (lse_host != nullptr &&
+        cudaMemcpyAsync(lse_host + static_cast<size_t>(h0) * N, dlse, static_cast<size_t>(nh) * N * 4,
+                        cudaMemcpyDeviceToHost, hp->s_out) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaEventRecord(hp->out_done[i], hp->s_out) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  // the call completes on `stream` once every result has reached the host
+  for (int i = 0; i < 2 && i < n_chunks; ++i)
+    if (cudaStreamWaitEvent(s, hp->out_done[i], 0) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}

@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
                                   "attn_status_string", "attn_debug_set_fault",
                                   "attn_fwd_noalloc", "attn_fwd_strided", "attn_bwd",
                                   "attn_bwd_workspace_bytes", "attn_fwd_splitkv",
-                                  "attn_fwd_splitkv_workspace_bytes", "attn_fwd_splitkv_auto_splits"])
+                                  "attn_fwd_splitkv_workspace_bytes", "attn_fwd_splitkv_auto_splits",
+                                  "attn_fwd_host", "attn_fwd_host_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -178,6 +179,30 @@ def test_splitkv_validation(lib):
     assert call(dtype=5) == binding.ATTN_ERR_UNSUPPORTED
     assert call(o=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
     assert call(lse=GOOD + 2) == binding.ATTN_ERR_MISALIGNED
+
+
+def test_host_forward_validation(lib):
+    F = lib.attn_fwd_host
+    ws = lib.attn_fwd_host_workspace_bytes(1, 8, 256, 64)
+    # two slots of (q, k, v, o) for ceil(8 / 8) = 1 head, plus LSE, 256-byte rounded
+    assert ws == 2 * (4 * 1 * 256 * 64 * 2 + 1 * 256 * 4)
+    assert lib.attn_fwd_host_workspace_bytes(4, 16, 100, 64) == 2 * (4 * 8 * 100 * 64 * 2 + 3328)
+    assert lib.attn_fwd_host_workspace_bytes(1, 1, 0, 64) == 0
+
+    def call(**kw):
+        a = dict(q=GOOD, k=GOOD, v=GOOD, o=GOOD, lse=None, B=1, H=8, N=256, d=64, scale=0.125, causal=0, dtype=0,
+                 ws=GOOD, ws_bytes=ws)
+        a.update(kw)
+        return F(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"],
+                 a["dtype"], a["ws"], a["ws_bytes"], None)
+
+    assert call(q=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(ws=None) == binding.ATTN_ERR_INVALID_ARG
+    assert call(ws_bytes=ws - 1) == binding.ATTN_ERR_INVALID_ARG
+    assert call(N=0) == binding.ATTN_ERR_INVALID_ARG
+    assert call(d=264) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(dtype=3) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(ws=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
 
 
 def test_debug_hook_validation(lib):
