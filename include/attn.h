@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1,  /* null pointer, size < 1, overflow, bad scale  */
-  ATTN_ERR_UNSUPPORTED = 2,  /* head dim or dtype this build does not handle */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head dim or dtype the library does not handle */
   ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned             */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed          */
   ATTN_ERR_TIMEOUT = 5       /* a kernel wait ran out (read after sync)       */
@@ -130,7 +130,7 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
  *                rotated).
  *   q_descale, k_descale, v_descale : [B][H][ceil(N/128)] fp32 factors.
  *   o   : [B][H][N][d] bf16, written.   lse : [B][H][N] fp32 or NULL.
- *   d   : 128 in this build (64 -> ATTN_ERR_UNSUPPORTED).
+ *   d   : 128 (64 -> ATTN_ERR_UNSUPPORTED).
  *   v_transpose : 0 = feed V to the tensor core MN-major, straight from the
  *                 TMA tile; 1 = transpose each V tile in shared memory to
  *                 K-major first (the pages' layout step; sm_100a accepts
