@@ -280,8 +280,8 @@ int attn_fwd_splitkv_auto_splits(int B, int H, int Nq, int Nk);
 
 /*
  * attn_fwd_host -- attn_fwd on HOST buffers, the transfers overlapped with
- * the computation: the B*H heads are processed in chunks (about an eighth
- * of the heads each) through two device slots in `workspace`; the
+ * the computation: the B*H heads are processed in chunks (about a
+ * sixteenth of the heads each) through two device slots in `workspace`; the
  * host-to-device copies of chunk c+1 (one internal stream) and the
  * device-to-host copies of chunk c-1 (another) run while chunk c computes on
  * `stream`.  One cudaMemcpyAsync per tensor and chunk.

@@ -184,9 +184,10 @@ def test_splitkv_validation(lib):
 def test_host_forward_validation(lib):
     F = lib.attn_fwd_host
     ws = lib.attn_fwd_host_workspace_bytes(1, 8, 256, 64)
-    # two slots of (q, k, v, o) for ceil(8 / 8) = 1 head, plus LSE, 256-byte rounded
+    # two slots of (q, k, v, o) for one head (fewer than 16 heads), plus LSE, 256-byte rounded
     assert ws == 2 * (4 * 1 * 256 * 64 * 2 + 1 * 256 * 4)
-    assert lib.attn_fwd_host_workspace_bytes(4, 16, 100, 64) == 2 * (4 * 8 * 100 * 64 * 2 + 3328)
+    # 64 heads: chunks of ceil(64 / 16) = 4 heads
+    assert lib.attn_fwd_host_workspace_bytes(4, 16, 100, 64) == 2 * (4 * 4 * 100 * 64 * 2 + 1792)
     assert lib.attn_fwd_host_workspace_bytes(1, 1, 0, 64) == 0
 
     def call(**kw):
