@@ -119,14 +119,17 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
 // The fused kernel
 // ---------------------------------------------------------------------------
 // Register split (setmaxnreg, per warpgroup): 512 threads launch with 128
-// registers each; the TMA/MMA warpgroup gives 40 to the row warpgroups and
-// the dQ warpgroup, which holds a whole 128-column dQ tile
-// (88 + 136 + 136 + 152 = 4 * 128).
-constexpr int kBwdRegsLow = 88;
-constexpr int kBwdRegsRows = 136;
-constexpr int kBwdRegsDq = 152;
-static_assert(128 * kBwdRegsLow + 256 * kBwdRegsRows + 128 * kBwdRegsDq <= 512 * 128,
-              "register split exceeds the launch pool");
+// registers each.  d=128: the TMA/MMA warpgroup gives 40 to the row
+// warpgroups and the dQ warpgroup, which holds a whole 128-column dQ tile
+// (88 + 136 + 136 + 152 = 4 * 128).  d=64: the MMA issuer runs the look-ahead
+// order (below) and keeps 112, the row warpgroups 128, the dQ warpgroup 144.
+template <int D>
+struct BwdRegs {
+  static constexpr int kLow = D == 64 ? 112 : 88;
+  static constexpr int kRows = D == 64 ? 128 : 136;
+  static constexpr int kDq = D == 64 ? 144 : 152;
+  static_assert(128 * kLow + 256 * kRows + 128 * kDq <= 512 * 128, "register split exceeds the launch pool");
+};
 
 template <typename E, int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_constant__ BwdParams p) {
@@ -166,6 +169,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   constexpr int kColS = Cfg::kColS, kColDP = Cfg::kColDP, kColDV = Cfg::kColDV, kColDK = Cfg::kColDK;
   constexpr int kColDQ = Cfg::kColDQ;
   constexpr int kPk = 32;            // packed P^T / dS^T start 32 columns into S^T / dP^T
+  // Look-ahead order (d=64, where dQ has columns of its own): S^T of the next
+  // tile is issued right after dV of this one, into the columns dV has just
+  // read, so the row warpgroups find it done when they finish dS.  At d=128,
+  // S^T of the next tile follows dQ instead, where it covers the load of dQ
+  // out of the columns the next dP^T takes (measured: look-ahead -10 % at
+  // d=128, +12-17 % at d=64).
+  constexpr bool kAhead = !Cfg::kDqShared;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -204,7 +214,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
   auto key_tile = [&](int blk) { return CAUSAL ? n_t - 1 - blk : blk; };
 
   if (warp < 4) {
-  reg_dealloc<kBwdRegsLow>();
+  reg_dealloc<BwdRegs<D>::kLow>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -293,6 +303,23 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         tc_fence_after();
         return r;
       };
+      // look-ahead order only: S^T and dP^T of tile t
+      auto issue_st = [&](uint32_t t) -> bool {
+        const uint32_t sq = t % SQ;
+        if (!mbar_wait(q_full + sq, (t / SQ) & 1, p.status, abort_flag, kWhereKvFull, lim)) return false;
+        tc_fence_after();
+        kmajor(kColS, dKd, dQk + ((sq * Cfg::kTileBytes) >> 4));
+        mma_commit(s_full);
+        return true;
+      };
+      auto issue_dpt = [&](uint32_t t) -> bool {
+        const uint32_t sd = t % SD;
+        if (!mbar_wait(do_full + sd, (t / SD) & 1, p.status, abort_flag, kWhereKvFull, lim)) return false;
+        tc_fence_after();
+        kmajor(kColDP, dVd, dDok + ((sd * Cfg::kTileBytes) >> 4));
+        mma_commit(dp_full);
+        return true;
+      };
       for (int k = 0; ok; ++k, ++unit_iter) {
         const int unit = sched_unit(k, p.snake);
         if (unit >= p.n_units) break;
@@ -304,6 +331,35 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         ok = mbar_wait(kv_full, unit_iter & 1, p.status, abort_flag, kWhereQFull, lim);
         tc_fence_after();
         if (!ok) break;
+        if constexpr (kAhead) {
+          // dV(t); S^T(t+1) into the columns dV(t) has just read; dK(t), dQ(t)
+          // (dQ in columns of its own, once dQ(t-1) is out); dP^T(t+1)
+          if (!(ok = issue_st(q_iter) && issue_dpt(q_iter))) break;
+          for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
+            const uint32_t sq = q_iter % SQ, sd = q_iter % SD;
+            const uint32_t qoff = (sq * Cfg::kTileBytes) >> 4, dooff = (sd * Cfg::kTileBytes) >> 4;
+            if (!(ok = mbar_wait(pt_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
+            tc_fence_after();
+            accum(kColDV, kColS + kPk, dDomn + dooff, i > i0);   // dV += P^T dO_i
+            mma_commit(do_empty + sd);
+            if (i + 1 < n_t && !(ok = issue_st(q_iter + 1))) break;
+            if (!(ok = mbar_wait(p_ready, q_iter & 1, p.status, abort_flag, kWherePFull, lim))) break;
+            tc_fence_after();
+            accum(kColDK, kColDP + kPk, dQmn + qoff, i > i0);    // dK += dS^T Q_i
+            mma_commit(q_empty + sq);
+            if (!(ok = wait_dq_free())) break;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + kColDQ, dDS + ((kk * 16 * 128) >> 4), dKmn + ((kk * 16 * 128) >> 4), idesc_dq,
+                     kk > 0 ? 1u : 0u, false);
+            mma_commit(dq_full);
+            if (i + 1 < n_t && !(ok = issue_dpt(q_iter + 1))) break;
+          }
+          if (!ok) break;
+          mma_commit(acc_full);
+          mma_commit(kv_empty);
+          continue;
+        }
         for (int i = i0; i < n_t && ok; ++i, ++q_iter) {
           const uint32_t sq = q_iter % SQ, sd = q_iter % SD;
           if (!(ok = mbar_wait(q_full + sq, (q_iter / SQ) & 1, p.status, abort_flag, kWhereKvFull, lim))) break;
@@ -350,7 +406,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
     __syncwarp();
   }
   } else if (warp < 12) {
-    if (kBwdRegsRows > 128) reg_alloc<kBwdRegsRows>();
+    if constexpr (BwdRegs<D>::kRows > 128) reg_alloc<BwdRegs<D>::kRows>();
     // ------------------------------------------------------------- key rows
     const int half = (warp - 4) >> 2;          // queries 64*half .. 64*half+63
     const int quarter = warp & 3;
@@ -388,12 +444,12 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         // warpgroup's 64 queries, packed to 16 bits into columns
         // 32 + 32*half .. of S^T (inside the 64 columns it has just read) --
         // the A operand of dV, which starts as soon as both halves are in.
+        uint32_t pp[32];   // P of this warpgroup's 64 queries, 16-bit pairs
         {
           uint32_t sr[64];
           tmem_ld32(tS + (2 * half) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr));
           tmem_ld32(tS + (2 * half + 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
           tmem_wait_ld();
-          uint32_t pp[32];
 #pragma unroll
           for (int x4 = 0; x4 < 16; ++x4) {
             const float4 lv = reinterpret_cast<const float4*>(lse2 + half * 64)[x4];   // broadcast reads
@@ -429,8 +485,16 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
           const int cc = half == 0 ? 1 - n : 2 + n;
+          // P of queries 32cc .. 32cc+31: from phase 1's registers under the
+          // look-ahead order (S^T of the next tile may already overwrite its
+          // columns), else read back from TMEM
           uint32_t pr16[16], dr[32];
-          tmem_ld16(tS + kPk + cc * 16, pr16);
+          if constexpr (kAhead) {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) pr16[x] = pp[(cc - 2 * half) * 16 + x];
+          } else {
+            tmem_ld16(tS + kPk + cc * 16, pr16);
+          }
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
           uint32_t pd[16];
@@ -477,7 +541,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
       }
     }
   } else {
-    reg_alloc<kBwdRegsDq>();
+    reg_alloc<BwdRegs<D>::kDq>();
     // ------------------------------------------------------------ dQ rows
     // Thread = query row.  The whole dQ tile goes to registers (then the
     // next dP^T may overwrite the columns), then 32 x 32 fp32 boxes, staged
