@@ -576,7 +576,7 @@ def main():
     ap.add_argument("--steps", type=int, default=600)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--ref-budget", type=float, default=15.0,
+    ap.add_argument("--ref-budget", type=float, default=30.0,
                     help="seconds of CPU work per oracle sample")
     ap.add_argument("--ref-total", type=float, default=150.0,
                     help="seconds of CPU work for the whole reference arm")
