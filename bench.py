@@ -481,10 +481,10 @@ def run_ours(args, world, rank, local):
                             "pct_of_spec_bf16_peak": 100 * tf_c / SPEC_BF16_TFLOPS},
             "bf16_backward_noncausal": {"tflops": 2.5 * f_nc / (bwd_ms[(False, False)] * 1e-3) / 1e12,
                                         "ms": bwd_ms[(False, False)], "kernels_per_call": 3,
-                                        "path": "fused, dQ by fp32 atomic adds"},
+                                        "path": "fused, dQ summed by fp32 TMA reduce-add"},
             "bf16_backward_causal": {"tflops": 2.5 * flops(B, H, N, d, True) / (bwd_ms[(True, False)] * 1e-3) / 1e12,
                                      "ms": bwd_ms[(True, False)], "kernels_per_call": 3,
-                                     "path": "fused, dQ by fp32 atomic adds"},
+                                     "path": "fused, dQ summed by fp32 TMA reduce-add"},
             "bf16_backward_noncausal_deterministic": {
                 "tflops": 2.5 * f_nc / (bwd_ms[(False, True)] * 1e-3) / 1e12, "ms": bwd_ms[(False, True)],
                 "kernels_per_call": 2, "path": "dQ kernel then dK/dV kernel, no atomics"},

@@ -216,8 +216,9 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int deterministic);
  *                     ATTN_ERR_UNSUPPORTED.
  *   deterministic   : 0 -- fused path (three kernels): one pass over the key
  *                     tiles computes dK, dV and dQ; dQ is summed over key
- *                     tiles by fp32 atomic adds into the workspace, so its
- *                     last bits may differ from run to run (dK, dV do not).
+ *                     tiles by fp32 TMA reduce-adds (atomic in L2) into the
+ *                     workspace, so its last bits may differ from run to run
+ *                     (dK, dV do not).
  *                     1 -- two kernels (dQ, then dK/dV), no atomics, every
  *                     output bit-reproducible; recomputes S and dP, so it
  *                     does seven N x N x d products instead of five.

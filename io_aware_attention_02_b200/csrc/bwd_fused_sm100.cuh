@@ -1,7 +1,7 @@
 // Fused attention backward for sm_100a: one pass over the key tiles that
 // produces dK, dV and dQ together (five N x N x d products instead of the
 // seven of the two-kernel path), with dQ summed across key tiles by fp32
-// atomic adds.  Same gradients as bwd_sm100.cuh ("FlashAttention-3"
+// TMA reduce-adds (atomic in L2).  Same gradients as bwd_sm100.cuh ("FlashAttention-3"
 // explainer, droidorbit.com, definition Softmax(Q K^T / sqrt(d)) V, chain
 // rule):
 //
