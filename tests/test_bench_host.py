@@ -1,0 +1,60 @@
+"""Host-side pieces of bench.py that need no GPU: the clock-record summary
+and the CPU-baseline record (the oracle timed on a small sample)."""
+
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from io_aware_attention_02_b200 import inputs  # noqa: E402
+
+
+def test_clock_summary_median_max_and_reasons():
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "0, 1600, 1965, 900.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1620, 1965, 950.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 980.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = c.summary()
+    assert s == {"sm_mhz": 1620.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_clock_summary_flags_throttling_reasons():
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1200, 1965, 1000, 0x48, Active, Not Active, Active, Not Active"]
+    assert c.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_summary_without_samples():
+    c = bench.ClockSampler(0)
+    c.lines = []
+    assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_cpu_baseline_record_has_the_required_keys():
+    q, k, v = inputs.qkv(1, 2, 256, 64, seed=0)
+    out = bench.oracle_sample(q, k, v, False, budget_s=0.5)
+    for key in ("value", "unit", "cores", "kind", "sample"):
+        assert key in out, key
+    assert out["kind"] == "oracle" and out["unit"] == "TFLOP/s"
+    assert out["value"] > 0 and out["cores"] >= 1
+    assert out["single_thread"]["value"] > 0
+
+
+def test_cpu_baseline_parity_sample_against_given_outputs():
+    """With the oracle's own outputs passed in as the 'GPU' result, the
+    parity sample is exactly zero."""
+    from oracle import attention as A
+    q, k, v = inputs.qkv(1, 2, 128, 32, seed=1)
+    o, l = A.attention(q, k, v, 1 / 32 ** 0.5, False)
+    import torch
+    out = bench.oracle_sample(q, k, v, False, budget_s=0.2, gpu_out=(torch.from_numpy(o), torch.from_numpy(l)),
+                              single_thread=False)
+    assert out["parity_sample"] == {"max_abs_dO": 0.0, "rmse_dO": 0.0, "max_abs_dLSE": 0.0}
+    assert "single_thread" not in out
