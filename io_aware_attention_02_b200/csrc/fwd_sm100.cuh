@@ -548,6 +548,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
           mma_commit(kv_empty + (ik % S));
         }
         if (!ok) break;
+        // the unit's last S products are issued: Q may be replaced by the next
+        // unit's once they complete (the P.V products left do not read it)
+        mma_commit(q_empty);
         const uint32_t iv = base + 2 * (n1 - 1) + 1;
         const uint32_t vs = wait_v(iv, ok);
         if (!ok) break;
@@ -558,7 +561,6 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         if (!(ok = pv(1, vs, n1 - 1 > 0))) break;
         mma_commit(o_full + 1);
         release_v(vs);
-        mma_commit(q_empty);
         kv_iter += 2 * n1;
       }
       if (!ok) {
