@@ -128,7 +128,8 @@ def test_accuracy_vs_low_precision_baselines(lib):
     scales and Hadamard rotation is more accurate than a per-tensor FP8
     attention, and the fp16 kernel (fp32 statistics) more accurate than a
     standard fp16 attention that writes its softmax out in fp16.  The pages
-    report 2.6x and 1.7x; here only the direction is asserted."""
+    report 2.6x and 1.7x (baselines whose rounding they do not describe);
+    measured here 1.59x and 1.03x; only the direction is asserted."""
     from oracle import baselines as Bl
     N, d = 1024, 128
     scale = 1 / math.sqrt(d)
@@ -148,5 +149,9 @@ def test_accuracy_vs_low_precision_baselines(lib):
         o_ref16, _ = A.attention_head(q6, k6, v6, scale)
         e16.append(Bl.rmse(o16[0, h].double().cpu().numpy(), o_ref16))
         e16b.append(Bl.rmse(Bl.standard_fp16_attention(q6, k6, v6, scale), o_ref16))
+    ratio8 = float(np.mean(e8b) / np.mean(e8))
+    ratio16 = float(np.mean(e16b) / np.mean(e16))
+    print(f"RMSE ratios: per-tensor FP8 / ours {ratio8:.2f} (pages 2.6), standard fp16 / ours {ratio16:.2f} "
+          f"(pages 1.7)")
     assert np.mean(e8) < np.mean(e8b), (e8, e8b)
     assert np.mean(e16) < np.mean(e16b), (e16, e16b)
