@@ -68,6 +68,18 @@ attn_status_t device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Kernel attributes (the dynamic shared-memory opt-in) are set per device:
+// each launch helper keeps one flag per device in `done`.
+bool attr_needed(bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return true;
+  return !done[dev];
+}
+void attr_mark(bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
+}
+
 // Element strides of a [B][H][N][d] view over (batch, head, row); the head
 // dim is contiguous.
 struct Strides {
@@ -154,12 +166,12 @@ template <typename E, int D, bool CAUSAL, bool VT = false>
 attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<E, D>;
   auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL, VT>;
-  static bool attr_done = false;  // per instance; set once per process
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};  // per instance and device
+  if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
-    attr_done = true;
+    attr_mark(attr_done);
   }
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -176,12 +188,12 @@ template <typename E, bool CAUSAL>
 attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream) {
   using Cfg = attn::Fwd256Cfg;
   auto kern = attn::attn_fwd_sm100_d256_kernel<E, CAUSAL>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
-    attr_done = true;
+    attr_mark(attr_done);
   }
   p.n_qpairs = (p.N + 127) / 128;
   p.n_units = p.BH * p.n_qpairs;
@@ -271,12 +283,12 @@ attn_status_t launch_bwd(attn::BwdParams p, int sm_count, cudaStream_t stream) {
   using Cfg = attn::BwdCfg<D>;
   auto kq = attn::attn_bwd_dq_kernel<E, D, CAUSAL>;
   auto kkv = attn::attn_bwd_dkdv_kernel<E, D, CAUSAL>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kDqSmem) != cudaSuccess ||
         cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kKvSmem) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    attr_done = true;
+    attr_mark(attr_done);
   }
   p.n_units = p.BH * p.n_t;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
@@ -299,11 +311,11 @@ attn_status_t launch_bwd_fused(attn::BwdParams p, int sm_count, const void* o, c
                                cudaStream_t stream) {
   using Cfg = attn::FusedCfg<D>;
   auto kf = attn::attn_bwd_fused_kernel<E, D, CAUSAL>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    attr_done = true;
+    attr_mark(attr_done);
   }
   attn::attn_bwd_prep_kernel<E><<<p.BH * p.n_t, 256, 0, stream>>>(
       static_cast<const E*>(o), static_cast<const E*>(d_o), p.lse, p.rows, p.dq_acc, p.N, p.n_t, p.d_out);
@@ -335,11 +347,11 @@ template <typename E, int D, bool CAUSAL>
 attn_status_t launch_splitkv(const attn::SplitParams& p, int grid, void* o, float* lse, cudaStream_t stream) {
   using Cfg = attn::SplitCfg<D>;
   auto kern = attn::attn_splitkv_kernel<E, D, CAUSAL>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    attr_done = true;
+    attr_mark(attr_done);
   }
   kern<<<grid, Cfg::kThreads, Cfg::kSmem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
