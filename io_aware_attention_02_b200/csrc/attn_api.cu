@@ -399,6 +399,23 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
   return b;
 }
 
+// Persistent quantiser: kMinBlocks CTAs per SM, each with its ring of bulk
+// copies in dynamic shared memory.
+template <int D>
+attn_status_t launch_quant(const attn::QuantParams& p, int sm_count, cudaStream_t stream) {
+  using C = attn::QuantCfg<D>;
+  static bool attr_done[kMaxDevices] = {};
+  if (attr_needed(attr_done)) {
+    if (cudaFuncSetAttribute(attn::attn_quant_fp8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmem) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_mark(attr_done);
+  }
+  const int grid = p.total < C::kMinBlocks * sm_count ? p.total : C::kMinBlocks * sm_count;
+  attn::attn_quant_fp8_kernel<D><<<grid, 256, C::kSmem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -470,16 +487,22 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
   if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(descale) & 3u) != 0 ||
       (signs != nullptr && (reinterpret_cast<uintptr_t>(signs) & 3u) != 0))
     return ATTN_ERR_MISALIGNED;
-  const int nb = (N + 127) / 128;
-  const int grid = nb * B * H;
+  DeviceState* st = nullptr;
+  attn_status_t r = device_state(&st);
+  if (r != ATTN_OK) return r;
+  attn::QuantParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.x8 = static_cast<uint8_t*>(x8);
+  p.descale = descale;
+  p.signs = signs;
+  p.status = st->status;
+  p.wait_limit_ns = wait_limit_ns();
+  p.N = N;
+  p.n_blocks = (N + 127) / 128;
+  p.total = p.n_blocks * B * H;
+  p.hadamard = hadamard;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  auto* q8 = static_cast<uint8_t*>(x8);
-  if (d == 64)
-    attn::attn_quant_fp8_kernel<64><<<grid, 256, 0, s>>>(xb, q8, descale, signs, N, nb, hadamard);
-  else
-    attn::attn_quant_fp8_kernel<128><<<grid, 256, 0, s>>>(xb, q8, descale, signs, N, nb, hadamard);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return d == 64 ? launch_quant<64>(p, st->sm_count, s) : launch_quant<128>(p, st->sm_count, s);
 }
 
 attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_descale,

@@ -55,6 +55,32 @@ def test_quant_hadamard_close(lib, d, signed):
     assert np.all(np.abs(vals[diff] - t[diff]) <= step[diff])
 
 
+@pytest.mark.parametrize("d,B,H,N", [(128, 1, 16, 32768 + 40), (64, 2, 8, 16384)])
+def test_quant_ring_of_copies_sampled_heads(lib, d, B, H, N):
+    """Sizes whose blocks outnumber the resident CTAs many times over, so each
+    CTA cycles its ring of block copies several times: plain quantisation is
+    bit-exact with the oracle on sampled heads (ragged last block included),
+    and the rotated one agrees as in the small cases."""
+    x = torch.empty((B, H, N, d), dtype=torch.bfloat16)
+    for b in range(B):
+        for h in range(H):
+            x[b, h] = inputs.head_bf16(11, "k", b, h, N, d, outliers=True)
+    xc = x.cuda()
+    codes, desc = lib.quant_fp8(xc)
+    signs = inputs.hadamard_signs(d, seed=4)
+    codes_r, desc_r = lib.quant_fp8(xc, hadamard=True, signs=torch.from_numpy(signs))
+    torch.cuda.synchronize()
+    assert lib.last_status()[0] == 0
+    for b, h in [(0, 0), (B - 1, H // 2 + 1), (B - 1, H - 1)]:
+        xh = x[b:b + 1, h:h + 1].double().numpy()
+        c_ref, d_ref, _ = F.quantize_blocks(xh)
+        np.testing.assert_array_equal(desc[b:b + 1, h:h + 1].cpu().numpy(), d_ref)
+        np.testing.assert_array_equal(codes[b:b + 1, h:h + 1].cpu().numpy(), c_ref)
+    c_ref, d_ref, _ = F.quantize_blocks(x[B - 1:B, H - 1:H].double().numpy(), True, signs)
+    np.testing.assert_allclose(desc_r[B - 1:B, H - 1:H].cpu().numpy(), d_ref, rtol=2e-6)
+    assert (codes_r[B - 1:B, H - 1:H].cpu().numpy() != c_ref).mean() < 2e-3
+
+
 def _fp8_attention(lib, q, k, v, causal, hadamard, signs=None):
     sg = torch.from_numpy(signs) if signs is not None else None
     q8, qd = lib.quant_fp8(q.cuda(), hadamard=hadamard, signs=sg)
