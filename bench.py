@@ -248,7 +248,10 @@ def oracle_sample(q, k, v, causal, budget_s=15.0, gpu_out=None, single_thread=Tr
     out = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
            "sample": f"{len(rows)} query rows x {len(heads)} heads of B={B},H={H},N={N},d={d} "
                      f"{'causal' if causal else 'non-causal'} (numpy fp64, full keys)",
-           "seconds": dt}
+           "seconds": dt,
+           # every row costs the same here (all keys scored, then masked), so the
+           # whole workload's time is the per-row time times all B*H*N rows
+           "extrapolated_full_workload_s": dt / (len(heads) * len(rows)) * B * H * N}
     if single_thread and threadpool_limits is not None:
         rows1 = inputs.sample_rows(N, 64, seed=13)
         with threadpool_limits(limits=1):

@@ -45,6 +45,8 @@ def test_cpu_baseline_record_has_the_required_keys():
     assert out["kind"] == "oracle" and out["unit"] == "TFLOP/s"
     assert out["value"] > 0 and out["cores"] >= 1
     assert out["single_thread"]["value"] > 0
+    # the projection to the whole workload scales the measured rows up
+    assert out["extrapolated_full_workload_s"] >= out["seconds"] * 0.999
 
 
 def test_cpu_baseline_parity_sample_against_given_outputs():
