@@ -298,9 +298,10 @@ int attn_fwd_splitkv_auto_splits(int B, int H, int Nq, int Nk);
  * the results are in host memory when `stream` has completed (synchronize
  * it before reading o_host / lse_host).  The copies start after the work
  * already queued on `stream`.  The library keeps two internal streams and
- * six events per device (created on first use); concurrent calls on one
- * device from several host threads are not supported.  Outputs are
- * bit-identical to attn_fwd on the same inputs.
+ * seven events per device (created on first use, kept until exit); calls on
+ * one device from several host threads take turns while they enqueue, and
+ * their copies share the two internal streams.  Outputs are bit-identical
+ * to attn_fwd on the same inputs.
  */
 attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                             float* lse_host, int B, int H, int N, int d, float scale, int causal, int dtype,

@@ -794,6 +794,7 @@ extern "C" attn_status_t attn_fwd_splitkv(const void* q, const void* k, const vo
 namespace {
 
 struct HostPipe {
+  std::mutex mu;  // held while a call enqueues on the shared streams and events
   bool ready = false;
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t start = nullptr, in_done[2] = {nullptr, nullptr}, comp_done[2] = {nullptr, nullptr},
@@ -858,6 +859,9 @@ extern "C" attn_status_t attn_fwd_host(const void* q_host, const void* k_host, c
   if (workspace_bytes < 2 * slot) return ATTN_ERR_INVALID_ARG;
   HostPipe* hp = nullptr;
   if ((r = host_pipe(&hp)) != ATTN_OK) return r;
+  // Calls from several host threads take turns enqueueing: each event wait
+  // below must see the record made by the same call.
+  std::lock_guard<std::mutex> pipe_lock(hp->mu);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t row_bytes = static_cast<size_t>(N) * d * 2;    // one head of one tensor
   const size_t t_bytes = static_cast<size_t>(chunk) * row_bytes;
