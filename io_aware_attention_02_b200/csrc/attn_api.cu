@@ -1,6 +1,7 @@
 // C ABI of libattn_sm100.so (declared in include/attn.h): argument
 // validation, TMA descriptor construction, kernel selection and launch.
 // Host code only marshals; every step of the attention runs in the kernels.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -69,15 +70,19 @@ attn_status_t device_state(DeviceState** out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Kernel attributes (the dynamic shared-memory opt-in) are set per device:
-// each launch helper keeps one flag per device in `done`.
-bool attr_needed(bool (&done)[kMaxDevices]) {
+// each launch helper keeps one flag per device in `done`.  The flags are
+// atomic so that calls from several host threads may race on them; the worst
+// case is setting the same attribute twice.
+using AttrFlags = std::atomic<bool>[kMaxDevices];
+bool attr_needed(AttrFlags& done) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return true;
-  return !done[dev];
+  return !done[dev].load(std::memory_order_acquire);
 }
-void attr_mark(bool (&done)[kMaxDevices]) {
+void attr_mark(AttrFlags& done) {
   int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices)
+    done[dev].store(true, std::memory_order_release);
 }
 
 // Element strides of a [B][H][N][d] view over (batch, head, row); the head
@@ -166,7 +171,7 @@ template <typename E, int D, bool CAUSAL, bool VT = false>
 attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<E, D>;
   auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL, VT>;
-  static bool attr_done[kMaxDevices] = {};  // per instance and device
+  static AttrFlags attr_done;  // per instance and device
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
@@ -188,7 +193,7 @@ template <typename E, bool CAUSAL>
 attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream) {
   using Cfg = attn::Fwd256Cfg;
   auto kern = attn::attn_fwd_sm100_d256_kernel<E, CAUSAL>;
-  static bool attr_done[kMaxDevices] = {};
+  static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
@@ -283,7 +288,7 @@ attn_status_t launch_bwd(attn::BwdParams p, int sm_count, cudaStream_t stream) {
   using Cfg = attn::BwdCfg<D>;
   auto kq = attn::attn_bwd_dq_kernel<E, D, CAUSAL>;
   auto kkv = attn::attn_bwd_dkdv_kernel<E, D, CAUSAL>;
-  static bool attr_done[kMaxDevices] = {};
+  static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kDqSmem) != cudaSuccess ||
         cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kKvSmem) != cudaSuccess)
@@ -311,7 +316,7 @@ attn_status_t launch_bwd_fused(attn::BwdParams p, int sm_count, const void* o, c
                                cudaStream_t stream) {
   using Cfg = attn::FusedCfg<D>;
   auto kf = attn::attn_bwd_fused_kernel<E, D, CAUSAL>;
-  static bool attr_done[kMaxDevices] = {};
+  static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -347,7 +352,7 @@ template <typename E, int D, bool CAUSAL>
 attn_status_t launch_splitkv(const attn::SplitParams& p, int grid, void* o, float* lse, cudaStream_t stream) {
   using Cfg = attn::SplitCfg<D>;
   auto kern = attn::attn_splitkv_kernel<E, D, CAUSAL>;
-  static bool attr_done[kMaxDevices] = {};
+  static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -404,7 +409,7 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
 template <int D>
 attn_status_t launch_quant(const attn::QuantParams& p, int sm_count, cudaStream_t stream) {
   using C = attn::QuantCfg<D>;
-  static bool attr_done[kMaxDevices] = {};
+  static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(attn::attn_quant_fp8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
