@@ -12,8 +12,10 @@ points to the extrema of the weighted error, repeat until the extrema
 equioscillate.  The fit runs in float64 and the result is rounded to fp32,
 the precision the kernel evaluates it in.
 
-This script is the source of the constants in csrc/fwd_sm100.cuh
-(kExp2Poly*); it prints them together with the achieved error bound.
+This script is the source of the coefficients of exp2_poly2 in
+csrc/fwd_sm100.cuh (degrees 3 and 2); it prints them together with the
+achieved error bound.  tests/test_exp2_poly.py checks that the kernel's
+literals are this fit rounded to fp32.
 """
 
 from __future__ import annotations
