@@ -58,6 +58,15 @@ def flops(B, H, N, d, causal):
     return f / 2 if causal else f
 
 
+def quant_roofline(B, H, N, d, n_tensors, ms, hbm_gbs):
+    """HBM roofline of the FP8 quantiser over `n_tensors` [B, H, N, d] bf16
+    tensors: algorithmic bytes = 2 read + 1 written per element plus one fp32
+    scale per 128-row block, over the measured time."""
+    nbytes = n_tensors * (3.0 * B * H * N * d + 4.0 * B * H * ((N + 127) // 128))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"quant_bytes": nbytes, "quant_GBs": gbs, "quant_frac_of_measured_hbm": gbs / hbm_gbs}
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("fwd_sm100.cuh", "ptx.cuh"):
@@ -499,6 +508,7 @@ def run_ours(args, world, rank, local):
             "fp8_e4m3_hadamard_noncausal": {
                 "tflops": tf_8, "ms": ms_8, "pct_of_spec_fp8_peak": 100 * tf_8 / SPEC_FP8_TFLOPS,
                 "quant_ms_qkv": ms_q,
+                **quant_roofline(B, H, N, d, 3, ms_q, float(peaks.get("hbm_gbs", 6650.0))),
                 "tflops_incl_quant": f_nc / ((ms_8 + ms_q) * 1e-3) / 1e12,
                 "tflops_v_transpose": f_nc / (ms_8t * 1e-3) / 1e12,
                 "inputs": "N(0,1) with 0.1% entries replaced by N(0,10^2)"},

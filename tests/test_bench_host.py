@@ -60,3 +60,13 @@ def test_cpu_baseline_parity_sample_against_given_outputs():
                               single_thread=False)
     assert out["parity_sample"] == {"max_abs_dO": 0.0, "rmse_dO": 0.0, "max_abs_dLSE": 0.0}
     assert "single_thread" not in out
+
+
+def test_quant_roofline_counts_bytes_per_element_and_block():
+    r = bench.quant_roofline(4, 16, 8192, 128, 3, 0.226, 6535.7)
+    elems = 4 * 16 * 8192 * 128
+    assert r["quant_bytes"] == 3 * (3 * elems + 4 * 4 * 16 * 64)
+    assert abs(r["quant_GBs"] - r["quant_bytes"] / 0.226e-3 / 1e9) < 1e-6
+    assert 0.40 < r["quant_frac_of_measured_hbm"] < 0.42
+    # a ragged last block still has its scale
+    assert bench.quant_roofline(1, 1, 129, 64, 1, 1.0, 1.0)["quant_bytes"] == 3 * 129 * 64 + 8
