@@ -4,11 +4,11 @@ gradients, called through the C ABI on seeded synthetic inputs.
 Tolerance, from the kernel's rounding: P and dS are rounded to the input
 dtype before the products that use them and every output is rounded to it
 once, so each gradient carries about two bf16 roundings (unit roundoff
-2^-9, i.e. ~1.1e-3 RMS relative each).  A CPU emulation of exactly those
-roundings on these inputs gives an RMSE of 2.2e-3 to 2.5e-3 of the
-gradient's RMS and a maximum error of 2.4e-3 to 4.2e-3 of its largest
-entry (N 300 to 1000, d 64 and 128, causal and not).  The bounds below are
-four and five times that.
+2^-9, i.e. ~1.1e-3 RMS relative each).  A CPU model of exactly those
+roundings (tests/test_backward_tolerance.py) gives an RMSE of 2.2e-3 to
+3.0e-3 of the gradient's RMS and a maximum error of 1.8e-3 to 6.5e-3 of its
+largest entry (N 300 to 1000, d 64 and 128, causal and not, both modes).
+The bounds below are about three times that.
 """
 
 import math
