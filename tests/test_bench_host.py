@@ -70,3 +70,32 @@ def test_quant_roofline_counts_bytes_per_element_and_block():
     assert 0.40 < r["quant_frac_of_measured_hbm"] < 0.42
     # a ragged last block still has its scale
     assert bench.quant_roofline(1, 1, 129, 64, 1, 1.0, 1.0)["quant_bytes"] == 3 * 129 * 64 + 8
+
+
+def _run_main(argv, env, capsys, monkeypatch):
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    monkeypatch.setattr(sys, "argv", ["bench.py", *argv])
+    bench.main()
+    return capsys.readouterr().out
+
+
+def test_reference_arm_other_ranks_exit_without_work(capsys, monkeypatch):
+    out = _run_main(["--impl", "reference", "--steps", "1", "--warmup", "3"], {"RANK": "1"}, capsys, monkeypatch)
+    assert out == ""
+
+
+def test_reference_arm_line_has_the_contract_keys(capsys, monkeypatch):
+    import json
+    out = _run_main(["--impl", "reference", "--steps", "1", "--warmup", "3", "--ref-budget", "0.2",
+                     "--ref-total", "1"], {"RANK": "0"}, capsys, monkeypatch)
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["config"]["workload"].startswith("B=4,H=16,N=8192,d=128")
