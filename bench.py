@@ -47,8 +47,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16/FP8 tensor peak"
 
 # DRAM bytes per launch of the bf16 d=128 non-causal kernel on the workload
-# above, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
-# (profiles/attn_fwd_bf16_d128_B4H16N8192.md), keyed by the sha256 of the
+# above, from the ncu DRAM capture of this kernel (`ncu --metrics
+# dram__bytes_read.sum,dram__bytes_write.sum`), keyed by the sha256 of the
 # kernel source it was measured on: reported only while the source is unchanged.
 TRAFFIC = {"5c96c7503f876e4f": 517090560}
 
@@ -309,6 +309,23 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def time_shape(B, H, N, d, causal, dev, steps, warmup, world):
+    """TFLOP/s of attn_fwd on one shape with timing-only inputs (torch.randn
+    bf16 on the device): a few steps, enough for a stable device time."""
+    from io_aware_attention_02_b200 import binding
+    g = torch.Generator(device=dev).manual_seed(0)
+    q, k, v = (torch.randn(B, H, N, d, device=dev, dtype=torch.bfloat16, generator=g) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    f = flops(B, H, N, d, causal)
+    n = max(3, min(steps, int(2e13 / f)))
+    ms = timed(lambda: binding.fwd(q, k, v, causal=causal, out=o, lse=lse), n, warmup, world) / n
+    return {"tflops": f / (ms * 1e-3) / 1e12, "ms": ms, "steps": n,
+            "pct_of_spec_bf16_peak": 100 * f / (ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS,
+            "shape": f"B={B},H={H},N={N},d={d},{'causal' if causal else 'non-causal'}",
+            "inputs": "torch.randn bf16 (timing only)"}
+
+
 def run_ours(args, world, rank, local):
     from io_aware_attention_02_b200 import binding
     binding.load()
@@ -359,6 +376,46 @@ def run_ours(args, world, rank, local):
             print(json.dumps({"metric": "attention bwd TFLOP/s (5 products, 10*B*H*N^2*d)",
                               "value": job_throughput(2.5 * f_nc, world, ms_b), "unit": "TFLOP/s",
                               "ms_per_step": ms_b, "steps": args.steps, "only": "bwd"}), flush=True)
+        return
+
+    if args.only in ("fp8", "quant"):
+        # profiler runs of the FP8 path at the headline shape: outlier inputs,
+        # Q and K rotated, 128 x d block scales
+        qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank_seed(rank), outliers=True))
+        signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
+        q8, qs = binding.quant_fp8(qo, hadamard=True, signs=signs)
+        k8, ks = binding.quant_fp8(ko, hadamard=True, signs=signs)
+        v8, vs = binding.quant_fp8(vo)
+        if args.only == "fp8":
+            def step_p():
+                binding.fwd_fp8(q8, k8, v8, qs, ks, vs, out=o, lse=lse)
+            fl = f_nc
+        else:
+            def step_p():
+                binding.quant_fp8(qo, hadamard=True, signs=signs, out=q8, descale=qs)
+                binding.quant_fp8(ko, hadamard=True, signs=signs, out=k8, descale=ks)
+                binding.quant_fp8(vo, out=v8, descale=vs)
+            fl = 0.0
+        ms_p = timed(step_p, args.steps, args.warmup, world) / args.steps
+        code, where = binding.last_status()
+        if code != 0:
+            raise RuntimeError(f"kernel status {code} at {where}")
+        if rank == 0:
+            print(json.dumps({"only": args.only, "ms_per_step": ms_p, "steps": args.steps,
+                              "tflops": fl / (ms_p * 1e-3) / 1e12 if fl else None,
+                              "quant_GBs": None if fl else 3 * (3.0 * B * H * N * d) / (ms_p * 1e-3) / 1e9}),
+                  flush=True)
+        return
+
+    if args.only in ("d64", "d256", "causal", "long"):
+        SB, SH, SN, Sd, sc = {"d64": (8, 16, 8192, 64, False), "d256": (2, 16, 8192, 256, False),
+                              "causal": (B, H, N, d, True), "long": (1, 32, 65536, 128, True)}[args.only]
+        r = time_shape(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
+        code, where = binding.last_status()
+        if code != 0:
+            raise RuntimeError(f"kernel status {code} at {where}")
+        if rank == 0:
+            print(json.dumps({"only": args.only, **r}), flush=True)
         return
 
     def step():
@@ -428,6 +485,19 @@ def run_ours(args, world, rank, local):
     kv_bytes_dec = 2 * DB * DH * DNk * d * 2
     del qdec, kdec, vdec, odec, ldec, wsd
 
+    # sequence-sweep points at 8K tokens (B*N = 16K, H = 16) for head dims 64
+    # and 256, and the long-context case; timing-only inputs (torch.randn)
+    shape_var = {}
+    for name, (SB, SH, SN, Sd, sc) in {
+            "bf16_d64_B2H16N8192": (2, 16, 8192, 64, False), "bf16_d64_B2H16N8192_causal": (2, 16, 8192, 64, True),
+            "bf16_d256_B2H16N8192": (2, 16, 8192, 256, False),
+            "bf16_d256_B2H16N8192_causal": (2, 16, 8192, 256, True),
+            "bf16_long_B1H32N65536_d128_causal": (1, 32, 65536, 128, True)}.items():
+        shape_var[name] = time_shape(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
+    code, where = binding.last_status()
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} at {where}")
+
     # FP8 variant: outlier inputs, Hadamard rotation of Q and K, 128 x d block scales
     qo, ko, vo = (t.to(dev) for t in inputs.qkv(B, H, N, d, seed=rank_seed(rank), outliers=True))
     signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
@@ -489,6 +559,7 @@ def run_ours(args, world, rank, local):
                      "peak_source": f"{src} bf16_tflops (burst cuBLAS 8192^3)",
                      "algorithmic_flops_per_launch": f_nc, "kernel_source": khash},
         "variants": {
+            **shape_var,
             "bf16_causal": {"tflops": tf_c, "ms": ms_c,
                             "pct_of_spec_bf16_peak": 100 * tf_c / SPEC_BF16_TFLOPS},
             "bf16_backward_noncausal": {"tflops": 2.5 * f_nc / (bwd_ms[(False, False)] * 1e-3) / 1e12,
@@ -552,10 +623,11 @@ def run_sweep(args):
 
 def run_ablation(args):
     """The pages' ablation shape {B=4, N=8448, H=16, d=128}, non-causal, bf16:
-    attn_fwd (two query tiles per CTA in ping-pong, S over P in TMEM) against
-    the same attention through attn_fwd_splitkv with one split (one query
-    tile per CTA, S double-buffered in TMEM, no ping-pong between tiles).
-    Runs alternate A/B/A/B in one process; one JSON line with the medians."""
+    one kernel (attn_fwd) with its two query tiles in ping-pong (the tensor
+    core works on one tile while the other tile's softmax runs) and with the
+    tiles serialised by attn_debug_set_ablation(1) (no product overlaps a
+    softmax).  Runs alternate A/B/A/B in one process; one JSON line with the
+    medians."""
     from io_aware_attention_02_b200 import binding
     torch.cuda.set_device(0)
     B, H, N, d = 4, 16, 8448, 128
@@ -563,16 +635,23 @@ def run_ablation(args):
     q, k, v = (torch.randn(B, H, N, d, device="cuda", dtype=torch.bfloat16, generator=g) for _ in range(3))
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
-    ws = torch.empty(int(binding.lib().attn_fwd_splitkv_workspace_bytes(B, H, N, d, 1)), dtype=torch.uint8,
-                     device="cuda")
-    arms = {"pingpong_two_tiles": lambda: binding.fwd(q, k, v, out=o, lse=lse),
-            "one_tile_s_double_buffered": lambda: binding.fwd_splitkv(q, k, v, n_splits=1, out=o, lse=lse,
-                                                                      workspace=ws)}
+
+    def arm(mode):
+        def fn():
+            binding.fwd(q, k, v, out=o, lse=lse)
+        def run():
+            binding.debug_set_ablation(mode)
+            try:
+                return timed(fn, steps, 3, 1) / steps
+            finally:
+                binding.debug_set_ablation(0)
+        return run
+    arms = {"pingpong_two_tiles": arm(0), "serialised_tiles": arm(1)}
     res = {name: [] for name in arms}
     steps = max(5, args.steps // 20)
     for _ in range(4):
-        for name, fn in arms.items():
-            res[name].append(timed(fn, steps, 3, 1) / steps)
+        for name, run in arms.items():
+            res[name].append(run())
     code, where = binding.last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {code} at {where}")
@@ -594,10 +673,13 @@ def main():
     ap.add_argument("--ref-total", type=float, default=150.0,
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "main", "bwd", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "main", "bwd", "decode", "fp8", "quant", "d64", "d256", "causal",
+                                       "long"], default="all",
                     help="main: time only the bf16 non-causal step; bwd: only the fused bf16 "
                          "non-causal backward of the same workload; decode: only the split-KV decode "
-                         "variant (for profiler runs)")
+                         "variant; fp8 / quant: only the FP8 forward / the FP8 quantisation of Q, K, V; "
+                         "d64 (B=8, N=8K), d256 (B=2, N=8K), causal, long (B=1, H=32, N=64K causal): "
+                         "only that bf16 forward (for profiler runs)")
     ap.add_argument("--decode-nk", type=int, default=32768,
                     help="KV length of the --only decode run (smaller for profiler captures)")
     ap.add_argument("--sweep", action="store_true",

@@ -130,11 +130,12 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
  *                rotated).
  *   q_descale, k_descale, v_descale : [B][H][ceil(N/128)] fp32 factors.
  *   o   : [B][H][N][d] bf16, written.   lse : [B][H][N] fp32 or NULL.
- *   d   : 128 (64 -> ATTN_ERR_UNSUPPORTED).
+ *   d   : 64 or 128 (others -> ATTN_ERR_UNSUPPORTED).
  *   v_transpose : 0 = feed V to the tensor core MN-major, straight from the
  *                 TMA tile; 1 = transpose each V tile in shared memory to
  *                 K-major first (the pages' layout step; sm_100a accepts
- *                 either, both give identical results).
+ *                 either, both give identical results).  1 needs d = 128
+ *                 (ATTN_ERR_UNSUPPORTED at d = 64).
  * Scores use scale * q_descale * k_descale per (query block, key block);
  * P is rounded to e4m3 after multiplying by 256 * v_descale[j] / max_j
  * v_descale[j]; statistics are fp32 and l sums the unrounded P.
@@ -161,11 +162,14 @@ attn_status_t attn_last_status(void* stream, int* where);
  * allocation attn_fwd performs for its status word) at a point where
  * allocation is forbidden.
  *   Arguments, layout, validation, results and error codes are those of
- *   attn_fwd, for head dims 64 and 128 (256 returns ATTN_ERR_UNSUPPORTED
- *   here).  The only scratch the kernel needs -- the 16-byte record its
- *   bounded waits write on a timeout -- lives in a static 256-byte device
- *   array inside the library instead of memory the library allocates.  That
- *   need does not grow with B, H, N or d, so no size exceeds the 256-byte
+ *   attn_fwd, except that only d == 64 and d == 128 are accepted: every
+ *   other head dim (including 256 and the zero-padded sizes attn_fwd takes)
+ *   returns ATTN_ERR_UNSUPPORTED.  Outputs are bit-identical to attn_fwd's
+ *   for the same arguments (the same kernel and schedule run).
+ *   The only scratch the kernel needs -- the 16-byte record its bounded
+ *   waits write on a timeout -- lives in a static 256-byte device array
+ *   inside the library instead of memory the library allocates.  That need
+ *   does not grow with B, H, N or d, so no size exceeds the 256-byte
  *   maximum; every GPU that loads the library holds the array until exit.
  *   This entry point calls no cudaMalloc, cudaFree or allocating routine.
  *   Its first call on a device looks up the array's device address (with
@@ -173,12 +177,25 @@ attn_status_t attn_last_status(void* stream, int* where);
  *   Every call clears the record on `stream` before its launch.  All calls
  *   share the one array, so calls whose kernels overlap on the GPU (on
  *   different streams) race on it.  A wait that runs out is recorded in that
- *   shared record only: attn_last_status() does not see it, and the outputs
- *   of that call are undefined.
+ *   shared record, not in attn_fwd's status word: read it with
+ *   attn_noalloc_last_status(); the outputs of a call that timed out are
+ *   undefined.
  */
 attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int N, int d, float scale, int causal, int dtype,
                                void* stream);
+
+/*
+ * attn_noalloc_last_status -- attn_last_status for attn_fwd_noalloc:
+ * synchronises `stream`, then reads and clears the shared record of the
+ * current device (through a host copy; nothing is allocated).  Returns
+ * ATTN_OK or ATTN_ERR_TIMEOUT (a wait of the last noalloc launch ran out;
+ * its outputs are undefined), ATTN_ERR_CUDA on a CUDA error.  `where` (may
+ * be NULL) receives 2 ints: the barrier id and block index recorded with the
+ * error.  With noalloc calls in flight on several streams the record holds
+ * whichever error was written first since the last clear.
+ */
+attn_status_t attn_noalloc_last_status(void* stream, int* where);
 
 /*
  * attn_bwd_workspace_bytes -- size of the workspace attn_bwd needs for these
@@ -259,8 +276,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *             H, Nq, d, n_splits) bytes (with the split count actually used),
  *             16-byte aligned, owned by the caller, contents irrelevant:
  *             fp32 partial O_s [n_splits][B*H][Nq][d] then LSE_s.
- *   d       : a multiple of 8, at most 128 (64 and 128 natively, others
- *             zero-padded).
+ *   d       : a multiple of 8, at most 256 (64, 128 and 256 natively, others
+ *             zero-padded to the next of those).
  *   scale, dtype, stream: as for attn_fwd.
  * Two kernels on `stream` (splits, then the merge).  Rounding: each split as
  * attn_fwd (fp32 statistics, P rounded to the input dtype) with O_s kept in
@@ -322,6 +339,32 @@ const char* attn_status_string(attn_status_t s);
  * wait limit for that launch.  No device fault, trap or hang is involved.
  */
 attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms);
+
+/*
+ * attn_debug_set_ablation -- bench hook for the pages' ablation of the
+ * overlap between the softmax and the matmuls (quantum-bit repost "H100
+ * utilisation 75% ... FlashAttention-3", ablation paragraph).  While `mode`
+ * is 1, attn_fwd / attn_fwd_strided / attn_fwd_host calls with bf16 inputs
+ * and head dim 128 (native, not padded) run a variant of the kernel whose two
+ * query tiles are serialised: the tensor core waits until both tiles have
+ * turned S into P before any product of the next key tile, and both tiles'
+ * next S are published together, so no product overlaps a softmax.  Results
+ * are bit-identical to mode 0 (the same products and roundings in the same
+ * order); only the schedule differs.  Other dtypes and head dims return
+ * ATTN_ERR_UNSUPPORTED while the mode is 1; attn_fwd_noalloc and
+ * attn_fwd_fp8 ignore it.  Mode 0 (the default) restores the ping-pong
+ * schedule.  The setting is global to the process and stays until changed.
+ * Returns ATTN_ERR_INVALID_ARG for other modes.
+ */
+attn_status_t attn_debug_set_ablation(int mode);
+
+/*
+ * attn_debug_status_allocated -- test query: 1 if the current device's
+ * attn_fwd status word (the one allocation the library makes on first use of
+ * a device) exists, 0 if not, -1 on a CUDA error.  Lets a test check that
+ * attn_fwd_noalloc and attn_noalloc_last_status allocate nothing.
+ */
+int attn_debug_status_allocated(void);
 
 #ifdef __cplusplus
 }

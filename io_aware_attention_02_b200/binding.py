@@ -30,6 +30,9 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_debug_set_fault": (_I, [_I, _I]),
     "attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_noalloc_last_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
+    "attn_debug_status_allocated": (_I, []),
+    "attn_debug_set_ablation": (_I, [_I]),
     "attn_fwd_strided": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _F, _I, _I, _P]),
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P, ctypes.c_size_t, _P]),
@@ -324,6 +327,26 @@ def last_status(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
     code = load().attn_last_status(ctypes.c_void_p(s), where)
     return code, [where[0], where[1]]
+
+
+def noalloc_last_status(stream=None):
+    """(status code, [barrier id, block index]) of the record attn_fwd_noalloc
+    writes (the library's static device array); clears it."""
+    where = (ctypes.c_int * 2)()
+    s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    code = load().attn_noalloc_last_status(ctypes.c_void_p(s), where)
+    return code, [where[0], where[1]]
+
+
+def debug_status_allocated() -> int:
+    """1 if attn_fwd's status word exists on the current device, else 0."""
+    return int(load().attn_debug_status_allocated())
+
+
+def debug_set_ablation(mode: int):
+    """1: serialise the two query tiles of the 16-bit forward (no overlap of
+    softmax and matmuls); 0: the normal ping-pong schedule."""
+    _check("attn_debug_set_ablation", load().attn_debug_set_ablation(int(mode)))
 
 
 def debug_set_fault(mode: int, wait_limit_ms: int = 0):

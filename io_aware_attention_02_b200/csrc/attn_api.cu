@@ -30,6 +30,7 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 int g_fault_mode = 0;
 int g_fault_limit_ms = 0;
+int g_ablation = 0;   // attn_debug_set_ablation: 1 = serialised tiles in the bf16 d = 128 forward
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -104,7 +105,8 @@ bool strides_ok(const Strides& s, int d, int esize) {
 }
 
 // 4-D tiled map over (d, N, H, B) with the given strides: box = (box_cols,
-// 128, 1, 1), 128-byte swizzle; out-of-range rows and columns read as zero.
+// 128, 1, 1), 128-byte swizzle (64-byte when the box row is 64 bytes);
+// out-of-range rows and columns read as zero.
 attn_status_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize,
                        int B, int H, int N, int D, const Strides& st, int box_cols) {
   EncodeTiledFn enc = encode_fn();
@@ -115,8 +117,9 @@ attn_status_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType d
                            static_cast<cuuint64_t>(st.b) * esize};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), 128u, 1u, 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUtensorMapSwizzle swz = box_cols * esize == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -167,10 +170,10 @@ void set_schedule(attn::FwdParams* p, int causal, int n_blocks, int grid, double
 
 double kv_bytes_of(int BH, int N, int d, int esize) { return 2.0 * BH * N * d * esize; }
 
-template <typename E, int D, bool CAUSAL, bool VT = false>
+template <typename E, int D, bool CAUSAL, bool VT = false, bool SERIAL = false>
 attn_status_t launch_fwd(const attn::FwdParams& p, int grid, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<E, D>;
-  auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL, VT>;
+  auto kern = attn::attn_fwd_sm100_kernel<E, D, CAUSAL, VT, SERIAL>;
   static AttrFlags attr_done;  // per instance and device
   if (attr_needed(attr_done)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
@@ -208,6 +211,17 @@ attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Hands the one-shot test hook (attn_debug_set_fault) to a launch and
+// resets it.
+void take_fault_hook(attn::FwdParams* p) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  p->fault = g_fault_mode;
+  if (g_fault_mode != 0 && g_fault_limit_ms > 0)
+    p->wait_limit_ns = static_cast<unsigned long long>(g_fault_limit_ms) * 1000000ull;
+  g_fault_mode = 0;
+  g_fault_limit_ms = 0;
+}
+
 // Fills the fields shared by the 16-bit and FP8 launches.
 attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void* o, int BH, int H,
                           int N, float scale) {
@@ -223,13 +237,13 @@ attn_status_t fill_common(attn::FwdParams* p, DeviceState* st, float* lse, void*
   p->n_units = BH * p->n_qpairs;
   p->scale_log2 = scale * 1.4426950408889634f;
   p->wait_limit_ns = wait_limit_ns();
-  std::lock_guard<std::mutex> lock(g_mu);
-  p->fault = g_fault_mode;
-  if (g_fault_mode != 0 && g_fault_limit_ms > 0)
-    p->wait_limit_ns = static_cast<unsigned long long>(g_fault_limit_ms) * 1000000ull;
-  g_fault_mode = 0;
-  g_fault_limit_ms = 0;
+  take_fault_hook(p);
   return ATTN_OK;
+}
+
+bool ablation_on() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_ablation != 0;
 }
 
 // 16-bit forward over strided [B][H][N][d] views (head dim contiguous).
@@ -273,6 +287,11 @@ attn_status_t fwd16(const void* q, const void* k, const void* v, void* o, float*
                     : launch_fwd256<__nv_bfloat16, false>(p, st->sm_count, s);
     return causal ? launch_fwd256<__half, true>(p, st->sm_count, s)
                   : launch_fwd256<__half, false>(p, st->sm_count, s);
+  }
+  if (ablation_on()) {   // bench hook: serialised query tiles, bf16 d = 128 only
+    if (dtype != ATTN_BF16 || dk != 128) return ATTN_ERR_UNSUPPORTED;
+    return causal ? launch_fwd<__nv_bfloat16, 128, true, false, true>(p, grid, s)
+                  : launch_fwd<__nv_bfloat16, 128, false, false, true>(p, grid, s);
   }
   if (dtype == ATTN_BF16)
     return dk == 64 ? launch_fwd_c<__nv_bfloat16, 64>(p, grid, causal, s)
@@ -404,8 +423,8 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
   return b;
 }
 
-// Persistent quantiser: kMinBlocks CTAs per SM, each with its ring of bulk
-// copies in dynamic shared memory.
+// Persistent quantiser: kMinBlocks CTAs of 128 threads per SM, each with its
+// ring of TMA block loads in dynamic shared memory.
 template <int D>
 attn_status_t launch_quant(const attn::QuantParams& p, int sm_count, cudaStream_t stream) {
   using C = attn::QuantCfg<D>;
@@ -417,7 +436,7 @@ attn_status_t launch_quant(const attn::QuantParams& p, int sm_count, cudaStream_
     attr_mark(attr_done);
   }
   const int grid = p.total < C::kMinBlocks * sm_count ? p.total : C::kMinBlocks * sm_count;
-  attn::attn_quant_fp8_kernel<D><<<grid, 256, C::kSmem, stream>>>(p);
+  attn::attn_quant_fp8_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -442,6 +461,13 @@ attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms) {
   std::lock_guard<std::mutex> lock(g_mu);
   g_fault_mode = mode;
   g_fault_limit_ms = wait_limit_ms;
+  return ATTN_OK;
+}
+
+attn_status_t attn_debug_set_ablation(int mode) {
+  if (mode < 0 || mode > 1) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_ablation = mode;
   return ATTN_OK;
 }
 
@@ -496,12 +522,17 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
   attn_status_t r = device_state(&st);
   if (r != ATTN_OK) return r;
   attn::QuantParams p{};
-  p.x = static_cast<const __nv_bfloat16*>(x);
-  p.x8 = static_cast<uint8_t*>(x8);
+  if ((r = make_map(&p.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, H, N, d, contiguous(H, N, d), 64)) !=
+      ATTN_OK)
+    return r;
+  // codes: one box spans a whole row of d bytes (64-byte swizzle at d = 64)
+  if ((r = make_map(&p.tm_x8, x8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, H, N, d, contiguous(H, N, d), d)) != ATTN_OK)
+    return r;
   p.descale = descale;
   p.signs = signs;
   p.status = st->status;
   p.wait_limit_ns = wait_limit_ns();
+  p.H = H;
   p.N = N;
   p.n_blocks = (N + 127) / 128;
   p.total = p.n_blocks * B * H;
@@ -521,7 +552,8 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   if (r != ATTN_OK) return r;
   if (v_transpose != 0 && v_transpose != 1) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (v_transpose && d != 128) return ATTN_ERR_UNSUPPORTED;   // the transposer handles 128-byte rows
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
   const uintptr_t a4 = reinterpret_cast<uintptr_t>(q_descale) | reinterpret_cast<uintptr_t>(k_descale) |
                        reinterpret_cast<uintptr_t>(v_descale) |
@@ -534,9 +566,10 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   attn::FwdParams p{};
   const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const Strides c8 = contiguous(H, N, d);
-  if ((r = make_map(&p.tm_q, q8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_k, k8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_v, v8, dt, 1, B, H, N, d, c8, 128)) != ATTN_OK) return r;
+  // one box spans a whole e4m3 row: 128 bytes (64-byte swizzle at d = 64)
+  if ((r = make_map(&p.tm_q, q8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
   p.q_desc = q_descale;
   p.k_desc = k_descale;
   p.v_desc = v_descale;
@@ -551,7 +584,8 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   if (v_transpose)
     return causal ? launch_fwd<__nv_fp8_e4m3, 128, true, true>(p, grid, s)
                   : launch_fwd<__nv_fp8_e4m3, 128, false, true>(p, grid, s);
-  return launch_fwd_c<__nv_fp8_e4m3, 128>(p, grid, causal, s);
+  return d == 64 ? launch_fwd_c<__nv_fp8_e4m3, 64>(p, grid, causal, s)
+                 : launch_fwd_c<__nv_fp8_e4m3, 128>(p, grid, causal, s);
 }
 
 }  // extern "C"
@@ -635,7 +669,7 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   p.n_units = BH * p.n_qpairs;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = wait_limit_ns();
-  p.fault = 0;
+  take_fault_hook(&p);
   p.d_out = d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the record keeps the previous call's contents: it must start at zero
@@ -647,6 +681,29 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
                    : launch_fwd_c<__nv_bfloat16, 128>(p, grid, causal, s);
   return d == 64 ? launch_fwd_c<__half, 64>(p, grid, causal, s)
                  : launch_fwd_c<__half, 128>(p, grid, causal, s);
+}
+
+extern "C" attn_status_t attn_noalloc_last_status(void* stream, int* where) {
+  NoAllocDevice* st = nullptr;
+  attn_status_t r = noalloc_device(&st);
+  if (r != ATTN_OK) return r;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};   // host copy of the record: no device memory involved
+  if (cudaMemcpy(h, st->scratch, kNoAllocStatusBytes, cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemset(st->scratch, 0, kNoAllocStatusBytes) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (where != nullptr) {
+    where[0] = h[1];
+    where[1] = h[2];
+  }
+  if (h[0] == 0) return ATTN_OK;
+  return h[0] == ATTN_ERR_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_debug_status_allocated(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_dev[dev].status != nullptr ? 1 : 0;
 }
 
 extern "C" size_t attn_bwd_workspace_bytes(int B, int H, int N, int d, int deterministic) {
@@ -744,7 +801,7 @@ extern "C" attn_status_t attn_fwd_splitkv(const void* q, const void* k, const vo
   if (causal && Nq > Nk) return ATTN_ERR_INVALID_ARG;   // every query must see at least one key
   if (n_splits < 0) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d > 128 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (d > 256 || (d % 8) != 0) return ATTN_ERR_UNSUPPORTED;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
   const void* p16[] = {q, k, v, o, workspace};
   for (const void* x : p16)
@@ -782,12 +839,14 @@ extern "C" attn_status_t attn_fwd_splitkv(const void* q, const void* k, const vo
   p.wait_limit_ns = wait_limit_ns();
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool d64 = d <= 64;
+  const int dk = d <= 64 ? 64 : (d <= 128 ? 128 : 256);
   if (dtype == ATTN_BF16)
-    return d64 ? launch_splitkv_c<__nv_bfloat16, 64>(p, grid, causal, o, lse, s)
-               : launch_splitkv_c<__nv_bfloat16, 128>(p, grid, causal, o, lse, s);
-  return d64 ? launch_splitkv_c<__half, 64>(p, grid, causal, o, lse, s)
-             : launch_splitkv_c<__half, 128>(p, grid, causal, o, lse, s);
+    return dk == 64    ? launch_splitkv_c<__nv_bfloat16, 64>(p, grid, causal, o, lse, s)
+           : dk == 128 ? launch_splitkv_c<__nv_bfloat16, 128>(p, grid, causal, o, lse, s)
+                       : launch_splitkv_c<__nv_bfloat16, 256>(p, grid, causal, o, lse, s);
+  return dk == 64    ? launch_splitkv_c<__half, 64>(p, grid, causal, o, lse, s)
+         : dk == 128 ? launch_splitkv_c<__half, 128>(p, grid, causal, o, lse, s)
+                     : launch_splitkv_c<__half, 256>(p, grid, causal, o, lse, s);
 }
 
 // ---------------------------------------------------------------------------

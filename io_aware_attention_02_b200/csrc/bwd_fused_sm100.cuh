@@ -450,6 +450,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           tmem_ld32(tS + (2 * half) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr));
           tmem_ld32(tS + (2 * half + 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
           tmem_wait_ld();
+          tmem_reg_fence(sr);
 #pragma unroll
           for (int x4 = 0; x4 < 16; ++x4) {
             const float4 lv = reinterpret_cast<const float4*>(lse2 + half * 64)[x4];   // broadcast reads
@@ -472,6 +473,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           tmem_st32(tS + kPk + half * 32, pp);
         }
         tmem_wait_st();
+        tmem_reg_fence(pp);
         tc_fence_before();
         mbar_arrive(pt_ready);
         w = mbar_wait(dp_full, t & 1, p.status, abort_flag, kWhereSFull, lim);
@@ -497,6 +499,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
           }
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
+          if constexpr (!kAhead) tmem_reg_fence(pr16);
+          tmem_reg_fence(dr);
           uint32_t pd[16];
 #pragma unroll
           for (int x4 = 0; x4 < 8; ++x4) {
@@ -517,8 +521,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
             *reinterpret_cast<uint4*>(ds_row + ((g ^ sw) << 4)) =
                 make_uint4(pd[4 * gg], pd[4 * gg + 1], pd[4 * gg + 2], pd[4 * gg + 3]);
           }
+          tmem_wait_st();   // the TMEM store reads pd asynchronously; the next chunk reuses it
+          tmem_reg_fence(pd);
         }
-        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_ready);
@@ -537,6 +542,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
         uint32_t rr[32];
         tmem_ld32(tA + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
         tmem_wait_ld();
+        tmem_reg_fence(rr);
         if (key_ok) store_row32<T>(dst, cc * 32, p.d_out, rr, mul);
       }
     }
@@ -568,6 +574,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_fused_kernel(const __grid_con
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tDQ + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(rr + cc * 32));
         tmem_wait_ld();
+        tmem_reg_fence(rr);
         tc_fence_before();
         mbar_arrive(dq_empty);
         const int row0 = i * 128 + quarter * 32;

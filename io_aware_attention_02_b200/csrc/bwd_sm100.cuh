@@ -309,6 +309,8 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
           tmem_ld32(tS + cc * 32, sr);
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
+          tmem_reg_fence(sr);
+          tmem_reg_fence(dr);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -323,6 +325,8 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
             pk[i] = pack2<T>(ds2[0], ds2[1]);
           }
           tmem_st16(tS + cc * 16, pk);
+          tmem_wait_st();   // the store reads pk asynchronously; the next chunk reuses it
+          tmem_reg_fence(pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -338,6 +342,7 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
         uint32_t rr[32];
         tmem_ld32(tDQ + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
         tmem_wait_ld();
+        tmem_reg_fence(rr);
         if (valid_row) store_row32<T>(drow, cc * 32, p.d_out, rr, p.scale);
       }
     }
@@ -552,6 +557,8 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
           tmem_ld32(tS + cc * 32, sr);
           tmem_ld32(tDP + cc * 32, dr);
           tmem_wait_ld();
+          tmem_reg_fence(sr);
+          tmem_reg_fence(dr);
           uint32_t pp[16], pd[16];
 #pragma unroll
           for (int ii = 0; ii < 16; ++ii) {
@@ -570,6 +577,9 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
           }
           tmem_st16(tS + cc * 16, pp);
           tmem_st16(tDP + cc * 16, pd);
+          tmem_wait_st();   // the stores read pp, pd asynchronously; the next chunk reuses them
+          tmem_reg_fence(pp);
+          tmem_reg_fence(pd);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -592,6 +602,7 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
           uint32_t rr[32];
           tmem_ld32(tA + cc * 32, rr);   // every lane loads (warp-wide); rows past N do not store
           tmem_wait_ld();
+          tmem_reg_fence(rr);
           if (valid) store_row32<T>(dst, cc * 32, p.d_out, rr, mul);
         }
       }

@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
         }
         tmem_wait_ld();
+        tmem_reg_fence(s);
         const int key0 = j * 128;
         const bool need_mask = (CAUSAL && key0 + 127 > qt * 128) || (key0 + 128 > p.N);
         if (need_mask) {
@@ -313,14 +314,18 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
               uint32_t r[32];
               tmem_ld32(tO + cc * 32, r);
               tmem_wait_ld();
+              tmem_reg_fence(r);
 #pragma unroll
               for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
               tmem_st32(tO + cc * 32, r);
+              tmem_wait_st();     // the store reads r asynchronously
+              tmem_reg_fence(r);
             }
           }
         }
         tmem_st32(tS, pk0);
         tmem_wait_st();
+        tmem_reg_fence(pk0);
         tc_fence_before();
         mbar_arrive(p_full + 0);
         sum += need_mask ? exp_pack_half<false, T, false>(s, 1, c, -m, 1.0f, tS)
@@ -352,6 +357,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         uint32_t r[32];
         tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
+        tmem_reg_fence(r);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)

@@ -100,9 +100,14 @@ struct FwdParams {
 template <typename E, int D>
 struct FwdCfg {
   static constexpr int kTileRows = 128;
-  static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
-  static constexpr int kChunkCols = 128 / Elem<E>::kBytes;
-  static constexpr int kChunks = D * Elem<E>::kBytes / 128;
+  // A tile is kChunks column chunks of 128 rows x kSwz bytes, each laid out
+  // with a kSwz-byte swizzle: 128 bytes, or 64 where a whole row is 64 bytes
+  // (e4m3 at head dim 64).
+  static constexpr int kRowBytes = D * Elem<E>::kBytes;
+  static constexpr int kSwz = kRowBytes >= 128 ? 128 : 64;
+  static constexpr int kChunkBytes = 128 * kSwz;
+  static constexpr int kChunkCols = kSwz / Elem<E>::kBytes;
+  static constexpr int kChunks = kRowBytes / kSwz;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStages = (kTileBytes <= 16384) ? 8 : 4;
   static constexpr int kKeysPerMma = 32 / Elem<E>::kBytes;  // 32 bytes of K per tcgen05.mma
@@ -210,7 +215,9 @@ constexpr int kPolyPairsPer8 = 1;
 
 // P = 2^(s*c - m) for one half (64 keys, h = 0 or 1) of a 128-key row:
 // packed to 16-bit pairs (or e4m3 quads, after the gain) and written over the
-// row's S columns in TMEM (32 columns per half at 16 bit, 16 at e4m3).
+// row's S columns in TMEM (32 columns per half at 16 bit, 16 at e4m3).  The
+// store has completed when it returns (tcgen05.st reads its source registers
+// asynchronously: they must not be reused before tcgen05.wait::st).
 // Returns the fp32 sum of the unrounded P of that half.
 template <bool kF8, typename T, bool kPoly>
 __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, float c, float neg_m,
@@ -229,6 +236,8 @@ __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, flo
       pk[i] = pack2<T>(pr.x, pr.y);
     }
     tmem_st32(tS + 32 * h, pk);
+    tmem_wait_st();
+    tmem_reg_fence(pk);
   } else {
     const float2 g2 = make_float2(pgain, pgain);
     uint32_t pk[16];
@@ -246,6 +255,8 @@ __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, flo
       pk[i] = pack4_e4m3(g0.x, g0.y, g1.x, g1.y);
     }
     tmem_st16(tS + 16 * h, pk);
+    tmem_wait_st();
+    tmem_reg_fence(pk);
   }
   const float2 a = __fadd2_rn(acc[0], acc[1]);
   return a.x + a.y;
@@ -301,7 +312,10 @@ constexpr int kRegsLow = 104;    // TMA + MMA warpgroup
 constexpr int kRegsHigh = 200;  // each softmax warpgroup
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch pool");
 
-template <typename E, int D, bool CAUSAL, bool VT = false>
+// SERIAL (the ablation of the overlap, 16-bit d = 128 only): the tensor core
+// waits for both tiles' P before any product of the next key tile, and both
+// tiles' S are published together, so no product overlaps a softmax.
+template <typename E, int D, bool CAUSAL, bool VT = false, bool SERIAL = false>
 __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   static_assert(!VT || (Elem<E>::kF8 && D == 128), "V transpose is the FP8 d=128 path");
   using Cfg = FwdCfg<E, D>;
@@ -435,10 +449,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       // Descriptors are built once and advanced by adding (byte offset >> 4)
       // to their start-address field (addresses stay below 256 KiB, so the
       // 14-bit field never carries).
-      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      constexpr int kSwz = Cfg::kSwz;
+      const uint64_t dQ = smem_desc_swz(smem_u32(sQ), 16, 8 * kSwz, kSwz);
+      const uint64_t dK = smem_desc_swz(smem_u32(sKV), 16, 8 * kSwz, kSwz);
       const uint64_t dV = VT ? smem_desc_sw128(smem_u32(sVt), 16, 1024)
-                             : smem_desc_sw128(smem_u32(sKV), Cfg::kChunkBytes, 1024);
+                             : smem_desc_swz(smem_u32(sKV), Cfg::kChunkBytes, 8 * kSwz, kSwz);
       uint32_t v_cnt = 0;   // V tiles consumed (VT: selects the transposed buffer and phase)
 
       auto issue_s = [&](int t, uint32_t kstage) {
@@ -446,9 +461,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         const uint64_t b0 = dK + static_cast<uint64_t>((kstage * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
-          // K-major, 128-byte swizzle: each product consumes 32 bytes of the
-          // head dim; four of them span one 128-byte chunk row.
-          const uint32_t off = ((kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32) >> 4;
+          // K-major, kSwz-byte swizzle: each product consumes 32 bytes of the
+          // head dim; four (128-byte swizzle) or two (64-byte) span one chunk
+          // row.
+          constexpr int kPerRow = kSwz / 32;   // products per swizzled row
+          const uint32_t off = ((kk / kPerRow) * Cfg::kChunkBytes + (kk % kPerRow) * 32) >> 4;
           mma_ss(tmem + Cfg::kColS + t * 128, a0 + off, b0 + off, idesc_s, kk > 0, kF8);
         }
       };
@@ -460,8 +477,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         for (int kk = h * kSteps; kk < (h + 1) * kSteps; ++kk) {
           // P_t: 128 rows x 128 keys packed in TMEM (32 bytes = 8 columns per
           // product).  V_j: MN-major (head dim contiguous), kKeysPerMma keys
-          // = kKeysPerMma rows of 128 bytes per product.
-          const uint32_t voff = VT ? ((kk * 32) >> 4) : ((kk * Cfg::kKeysPerMma * 128) >> 4);
+          // = kKeysPerMma swizzled rows of kSwz bytes per product.
+          const uint32_t voff = VT ? ((kk * 32) >> 4) : ((kk * Cfg::kKeysPerMma * kSwz) >> 4);
           mma_ts(tmem + Cfg::kColO + t * D, tmem + Cfg::kColS + t * 128 + kk * 8,
                  b0 + voff, idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
         }
@@ -476,6 +493,15 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
           issue_pv_half(t, vstage, h, acc);
         }
         ++p_cnt[t];
+        return true;
+      };
+      // Ablation (serial): wait until both tiles have published P(j-1)
+      // before any product of step j, so that the tensor core never runs
+      // while a softmax does (pv() then finds those phases complete).
+      auto wait_p_both = [&](bool has0) -> bool {
+        for (int t = has0 ? 0 : 1; t < 2; ++t)
+          for (int h = 0; h < 2; ++h)
+            if (!mbar_wait(p_full + 2 * t + h, p_cnt[t] & 1, p.status, abort_flag, kWherePFull, lim)) return false;
         return true;
       };
       auto wait_kv = [&](uint32_t idx) -> bool {
@@ -533,10 +559,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
           if (!(ok = wait_kv(ik))) break;
           const uint32_t vs = wait_v(iv, ok);
           if (!ok) break;
+          if (SERIAL && !(ok = wait_p_both(j <= n0))) break;
           if (j < n0) {
             if (!(ok = pv(0, vs, j - 1 > 0))) break;
             issue_s(0, ik % S);
-            mma_commit(s_full + 0);
+            if (!SERIAL) mma_commit(s_full + 0);
           } else if (j == n0) {
             if (!(ok = pv(0, vs, j - 1 > 0))) break;
             mma_commit(o_full + 0);
@@ -544,6 +571,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
           if (!(ok = pv(1, vs, j - 1 > 0))) break;
           release_v(vs);
           issue_s(1, ik % S);
+          if (SERIAL && j < n0) mma_commit(s_full + 0);   // both S published together
           mma_commit(s_full + 1);
           mma_commit(kv_empty + (ik % S));
         }
@@ -666,6 +694,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
         }
         tmem_wait_ld();
+        tmem_reg_fence(s);
 
         const int key0 = j * 128;
         const bool need_mask = (CAUSAL && key0 + 127 > qp * 256 + t * 128) || (key0 + 128 > p.N);
@@ -688,19 +717,24 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         // first half of P is published (its PV product accumulates into O_t).
         // The PV product of the previous key tile has completed: S_t(j) was
         // committed after it.
+        // (16 columns at a time: with the 128 scores live, wider chunks
+        // would spill)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld32(tO + cc * 32, r);
+#pragma unroll 1
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t r[16];
+            tmem_ld16(tO + cc * 16, r);
             tmem_wait_ld();
+            tmem_reg_fence(r);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tO + cc * 32, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st16(tO + cc * 16, r);
+            tmem_wait_st();       // the store reads r asynchronously; the next chunk reloads it
+            tmem_reg_fence(r);
           }
         }
         // P in two halves of 64 keys, each published as soon as it is in
-        // TMEM.  Masked tiles hold -inf scores, which only the MUFU path maps
+        // TMEM (exp_pack_half returns with its store complete).  Masked tiles hold -inf scores, which only the MUFU path maps
         // to an exact 0; unmasked tiles may send part of their exp2 work to
         // the FMA pipe.
         float sum = 0.f;
@@ -732,6 +766,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         uint32_t r[32];
         tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
+        tmem_reg_fence(r);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)

@@ -223,6 +223,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -249,6 +257,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// tcgen05.ld fills its destination registers asynchronously: they may be
+// read only after tcgen05.wait::ld, an ordering the compiler does not see (to
+// it the registers are defined by the load instruction itself).  Passing them
+// through an empty volatile asm placed after the wait makes every later use
+// read the values as they stand after the wait.
+template <int N>
+__device__ __forceinline__ void tmem_reg_fence(uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "eight registers per statement");
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]),
+                      "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_reg_fence(float (&r)[N]) {
+  static_assert(N % 8 == 0, "eight registers per statement");
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+f"(r[i]), "+f"(r[i + 1]), "+f"(r[i + 2]), "+f"(r[i + 3]), "+f"(r[i + 4]),
+                      "+f"(r[i + 5]), "+f"(r[i + 6]), "+f"(r[i + 7]));
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -260,6 +290,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const 
   asm volatile(
       "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
       ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// Tiled store of a shared-memory box to global memory, 4-D map, no
+// multicast; completion is tracked by this thread's bulk-async groups.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() {
@@ -285,16 +323,20 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // ----------------------------------------------------------------------------
 // Descriptors
 // ----------------------------------------------------------------------------
-// Shared-memory matrix descriptor for tcgen05 (version 1), 128-byte swizzle.
+// Shared-memory matrix descriptor for tcgen05 (version 1) with a 128-byte or
+// 64-byte swizzle (`swz` = 128 or 64: the span of one swizzled row).
 // `lbo` / `sbo` are byte offsets (multiples of 16).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+__device__ __forceinline__ uint64_t smem_desc_swz(uint32_t saddr, uint32_t lbo, uint32_t sbo, int swz) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
-  d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100
-  d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+  d |= static_cast<uint64_t>(1) << 46;                         // descriptor version for sm_100
+  d |= static_cast<uint64_t>(swz == 64 ? 4 : 2) << 61;         // SWIZZLE_64B : SWIZZLE_128B
   return d;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc_swz(saddr, lbo, sbo, 128);
 }
 
 // Instruction descriptor for kind::f16 / kind::f8f6f4, fp32 accumulator.

@@ -8,17 +8,24 @@
 // "FlashAttention-3 (HE)" (systems-analysis.info), "Technical innovations",
 // item 3.  The rotation leaves Q K^T unchanged because it is orthogonal.
 //
-// Pure streaming kernel: 2 bytes read and 1 byte written per element, bound
-// by HBM bandwidth.  Persistent CTAs (two or three per SM) walk the blocks of
-// 128 rows of one (batch, head) in a strided order.  A block is one
-// contiguous run of 128 * D bf16 values, so one thread copies it into shared
-// memory with a single bulk copy; a ring of kStages such copies per CTA keeps
-// bytes in flight while the CTA works on the oldest one.  Each row is handled
-// by D/8 threads holding 8 consecutive values: the fast Walsh-Hadamard
-// transform runs three butterfly stages in registers and the rest across
-// lanes with shuffles.  The block's amax needs every row, so the CTA meets at
-// one barrier per block; that barrier also tells the copying thread that the
-// block's buffer has been read and may be refilled.
+// Streaming kernel: 2 bytes read and 1 byte written per element, meant to run
+// at HBM bandwidth.  Persistent CTAs of 128 * D/64 threads (two or three per
+// SM) walk the blocks of 128 rows of one (batch, head) in a strided order.
+// Thread 0 keeps a ring of kStages blocks in flight: each block arrives by
+// TMA (tile loads of 64 columns x 128 rows, 128-byte swizzle, rows past N
+// zero-filled).  A thread owns 64 columns of one row (the two threads of a
+// d = 128 row are neighbouring lanes): it reads them from shared memory (the
+// swizzle spreads a warp's 16-byte reads over all banks), applies the signs
+// (a flip of the bf16 sign bits), runs the six butterfly stages of the fast
+// Walsh-Hadamard transform that stay inside its 64 values in registers and,
+// at d = 128, the last stage with its neighbour by one lane shuffle per
+// value; then it scales by 1/sqrt(D) and takes its amax.  The block's amax
+// needs every row, so the CTA meets at one barrier per block; that barrier
+// also tells thread 0 that the block's buffer has been read and may be
+// refilled.  Each thread then rounds its 64 values to e4m3 into one of two
+// shared-memory staging tiles (swizzled like the input, so a warp's 16-byte
+// writes spread over all banks), and thread 0 writes the block to global
+// memory with one TMA store (rows past N are clipped).
 #pragma once
 #include "ptx.cuh"
 
@@ -27,28 +34,37 @@ namespace attn {
 enum : int { kWhereQuantFull = 10 };
 
 struct QuantParams {
-  const __nv_bfloat16* x;   // [BH][N][D]
-  uint8_t* x8;              // [BH][N][D] e4m3 codes
+  CUtensorMap tm_x;         // 4-D map over x (D, N, H, B): box 64 x 128, 128-byte swizzle
+  CUtensorMap tm_x8;        // 4-D map over the codes (D, N, H, B): box D x 128, D-byte swizzle
   float* descale;           // [BH][n_blocks]
   const float* signs;       // [D] or nullptr
   int* status;
   unsigned long long wait_limit_ns;
-  int N, n_blocks, total;   // total = BH * n_blocks
+  int H, N, n_blocks, total;   // total = BH * n_blocks
   int hadamard;
 };
 
 template <int D>
 struct QuantCfg {
   static constexpr int kRows = 128;
-  static constexpr int kTileBytes = kRows * D * 2;
-  // 3 x 32 KiB per CTA and two CTAs per SM at D = 128; 4 x 16 KiB and three
-  // CTAs per SM at D = 64 (registers allow it there).
-  static constexpr int kStages = D == 64 ? 4 : 3;
+  static constexpr int kChunkBytes = kRows * 128;            // 64 bf16 columns x 128 rows
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  // input ring + two output staging tiles: 2 x 32 + 2 x 16 KiB per CTA and
+  // two CTAs per SM at D = 128; 3 x 16 + 2 x 8 KiB and three CTAs at D = 64
+  static constexpr int kStages = D == 64 ? 3 : 2;
   static constexpr int kMinBlocks = D == 64 ? 3 : 2;
-  static constexpr int kBarOff = kStages * kTileBytes;
+  static constexpr int kOutBytes = kRows * D;                // one block of codes
+  static constexpr int kTpr = D / 64;                        // threads per row
+  static constexpr int kThreads = 128 * kTpr;
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kOutOff = kStages * kTileBytes;     // [2] staging tiles
+  static constexpr int kBarOff = kOutOff + 2 * kOutBytes;
   static constexpr int kAbortOff = kBarOff + 64;
-  static constexpr int kRedOff = kBarOff + 128;             // float [2][8]
-  static constexpr int kSmem = kBarOff + 256;
+  static constexpr int kRedOff = kBarOff + 128;             // float [2][kWarps <= 8]
+  static constexpr int kSgnOff = kBarOff + 256;             // uint32 [D / 2]: sign bits per bf16 pair
+  static_assert(2 * kWarps * 4 <= 128, "amax slots overflow their region");
+  static constexpr int kSmem = kSgnOff + 2 * D + 1024;      // + alignment slack for the swizzle
   static_assert(kStages * 8 <= 64, "barriers overflow their slot");
 };
 
@@ -73,31 +89,31 @@ __device__ __forceinline__ uint32_t quant4_e4m3(const float* y, float s, float r
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, QuantCfg<D>::kMinBlocks) attn_quant_fp8_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks)
+    attn_quant_fp8_kernel(const __grid_constant__ QuantParams p) {
   using C = QuantCfg<D>;
-  constexpr int TPR = D / 8;              // threads per row
-  constexpr int RPP = 256 / TPR;          // rows per pass
-  constexpr int PASSES = 128 / RPP;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  auto* tiles = reinterpret_cast<__nv_bfloat16*>(smem);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle pattern
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   auto* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   auto* abort_flag = reinterpret_cast<volatile int*>(smem + C::kAbortOff);
   auto* red = reinterpret_cast<float*>(smem + C::kRedOff);
+  auto* sgn = reinterpret_cast<uint32_t*>(smem + C::kSgnOff);
+  uint8_t* out_tiles = smem + C::kOutOff;
 
   const int tid = threadIdx.x;
-  const int rip = tid / TPR;              // row within pass
-  const int seg = tid % TPR;              // 8-value segment within the row
+  const int r = tid / C::kTpr;            // row within the block
+  const int hc = tid % C::kTpr;           // 64-column chunk of that row
+  const int warp = tid >> 5;
 
-  // Block t = bh * n_blocks + blk: rows [128 blk, min(128 blk + 128, N)) of
-  // head bh, contiguous in memory.
+  // Block t = bh * n_blocks + blk: rows [128 blk, 128 blk + 128) of head bh.
   auto issue = [&](int t, int stage) {
-    const int blk = t % p.n_blocks;
-    const int rows = min(C::kRows, p.N - blk * C::kRows);
-    const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
-    const __nv_bfloat16* src = p.x + static_cast<size_t>(t / p.n_blocks) * p.N * D +
-                               static_cast<size_t>(blk) * C::kRows * D;
-    mbar_arrive_expect_tx(&full[stage], bytes);
-    bulk_load(tiles + static_cast<size_t>(stage) * C::kRows * D, src, bytes, &full[stage]);
+    const int bh = t / p.n_blocks, blk = t % p.n_blocks;
+    mbar_arrive_expect_tx(&full[stage], C::kTileBytes);
+#pragma unroll
+    for (int c = 0; c < C::kChunks; ++c)
+      tma_load_4d(smem + stage * C::kTileBytes + c * C::kChunkBytes, &p.tm_x, &full[stage], c * 64,
+                  blk * C::kRows, bh % p.H, bh / p.H);
   };
 
   if (tid == 0) {
@@ -105,17 +121,27 @@ __global__ void __launch_bounds__(256, QuantCfg<D>::kMinBlocks) attn_quant_fp8_k
     *abort_flag = 0;
     fence_barrier_init();
   }
+  // The signs as bf16 sign bits, one word per pair of elements: multiplying
+  // by -1 is flipping that bit of the packed input (exact).
+  if (tid < D / 2) {
+    uint32_t w = 0;
+    if (p.hadamard && p.signs != nullptr) {
+      if (p.signs[2 * tid] < 0.f) w |= 0x8000u;
+      if (p.signs[2 * tid + 1] < 0.f) w |= 0x80000000u;
+    }
+    sgn[tid] = w;
+  }
   __syncthreads();
   if (tid == 0) {
+    tma_prefetch_desc(&p.tm_x);
+    tma_prefetch_desc(&p.tm_x8);
     for (int s = 0; s < C::kStages; ++s) {
       const int t = blockIdx.x + s * gridDim.x;
       if (t < p.total) issue(t, s);
     }
   }
 
-  float sg[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) sg[i] = (p.hadamard && p.signs != nullptr) ? p.signs[seg * 8 + i] : 1.f;
+  const bool rot = p.hadamard != 0;
   const float norm = rsqrtf(static_cast<float>(D));
 
   int it = 0;
@@ -125,65 +151,67 @@ __global__ void __launch_bounds__(256, QuantCfg<D>::kMinBlocks) attn_quant_fp8_k
     const bool ok = mbar_wait(&full[stage], (it / C::kStages) & 1, p.status, abort_flag,
                               kWhereQuantFull, p.wait_limit_ns);
     const int row0 = (t % p.n_blocks) * C::kRows;
-    const __nv_bfloat16* tile = tiles + static_cast<size_t>(stage) * C::kRows * D;
 
-    float y[PASSES][8];
+    // this thread's 64 values from the swizzled tile (16-byte piece q of the
+    // 64-column chunk sits at piece q ^ (row % 8) of the row's 128 bytes)
+    float y[64];
+    const uint8_t* tile = smem + stage * C::kTileBytes + hc * C::kChunkBytes + r * 128;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (ok) raw = *reinterpret_cast<const uint4*>(tile + ((q ^ (r & 7)) << 4));
+      if (rot) {   // four words shared by all threads of a chunk: a broadcast read
+        const uint4 m = reinterpret_cast<const uint4*>(sgn)[hc * 8 + q];
+        raw.x ^= m.x; raw.y ^= m.y; raw.z ^= m.z; raw.w ^= m.w;
+      }
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = unpack2<__nv_bfloat16>(w[i]);
+        y[q * 8 + 2 * i] = f.x;
+        y[q * 8 + 2 * i + 1] = f.y;
+      }
+    }
+    if (rot) {
+      // fast Walsh-Hadamard transform, one rounding per output of each stage:
+      // the stages over the 6 low index bits inside this thread ...
+#pragma unroll
+      for (int h = 1; h < 64; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          if ((i & h) == 0) {
+            const float a = y[i], b = y[i | h];
+            y[i] = a + b;
+            y[i | h] = a - b;
+          }
+        }
+      }
+      // ... and at d = 128 the stage over index bit 6 with the neighbouring
+      // lane (lower chunk: y + other; upper chunk: other - y)
+      if constexpr (C::kTpr == 2) {
+        const float sg = hc == 0 ? 1.f : -1.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float other = __shfl_xor_sync(0xffffffffu, y[i], 1);
+          y[i] = fmaf(sg, y[i], other);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 64; ++i) y[i] *= norm;
+    }
     float amax = 0.f;
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int r = ps * RPP + rip;
-      if (ok && row0 + r < p.N) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(tile + r * D + seg * 8);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(h2[i]);
-          y[ps][2 * i] = f.x;
-          y[ps][2 * i + 1] = f.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[ps][i] = 0.f;
-      }
-      if (p.hadamard) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[ps][i] *= sg[i];
-        // butterflies over the 3 low index bits (inside this thread)
-#pragma unroll
-        for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if ((i & h) == 0) {
-              const float a = y[ps][i], b = y[ps][i | h];
-              y[ps][i] = a + b;
-              y[ps][i | h] = a - b;
-            }
-          }
-        }
-        // butterflies over the high index bits (across the row's lanes)
-#pragma unroll
-        for (int m = 1; m < TPR; m <<= 1) {
-          // lower lane: y + other; upper lane: other - y (one rounding each)
-          const float sgn = (seg & m) != 0 ? -1.f : 1.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float other = __shfl_xor_sync(0xffffffffu, y[ps][i], m);
-            y[ps][i] = fmaf(sgn, y[ps][i], other);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[ps][i] *= norm;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[ps][i]));
-    }
+    for (int i = 0; i < 64; i += 2) amax = fmax3(amax, fabsf(y[i]), fabsf(y[i + 1]));
 
     // Block amax.  The slots alternate between blocks: a warp writes slot
     // set (it & 1) again only two barriers later, after every warp has read it.
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    float* slots = red + (it & 1) * 8;
-    if ((tid & 31) == 0) slots[tid >> 5] = amax;
+    float* slots = red + (it & 1) * C::kWarps;
+    if ((tid & 31) == 0) slots[warp] = amax;
+    // staging tile (it & 1) was last stored two blocks ago: let that store
+    // finish reading it before anyone writes it again (the barrier below)
+    if (tid == 0) bulk_wait_group_read<1>();
     // Every thread has read this block's buffer once it passes the barrier;
     // a wait that gave up anywhere ends the loop in every thread.
     if (__syncthreads_or(!ok)) {
@@ -199,27 +227,39 @@ __global__ void __launch_bounds__(256, QuantCfg<D>::kMinBlocks) attn_quant_fp8_k
     }
     float bmax = slots[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) bmax = fmaxf(bmax, slots[w]);
+    for (int w = 1; w < C::kWarps; ++w) bmax = fmaxf(bmax, slots[w]);
     const float s = (bmax == 0.f) ? 1.0f : __fdiv_rn(bmax, 448.0f);
     if (tid == 0) p.descale[t] = s;
     // The bracket needs the reciprocal and the products to stay normal and
     // finite: a block scale far outside [2^-100, 2^100] takes the division.
     const bool fast = s >= 0x1p-100f && s <= 0x1p100f;
-    const float r = __frcp_rn(s);
-    const float r_lo = __fmul_rn(r, 1.f - 0x1p-20f), r_hi = __fmul_rn(r, 1.f + 0x1p-20f);
+    const float rc = __frcp_rn(s);
+    const float r_lo = __fmul_rn(rc, 1.f - 0x1p-20f), r_hi = __fmul_rn(rc, 1.f + 0x1p-20f);
 
-    uint8_t* out_blk = p.x8 + static_cast<size_t>(t / p.n_blocks) * p.N * D + static_cast<size_t>(row0) * D;
+    // this thread's 64 codes: 16-byte pieces hc*4 + g of the row, swizzled
+    // the way the TMA store reads them (the D-byte swizzle XORs the 16-byte
+    // piece index with address bits 7 and up: row % 8 for 128-byte rows,
+    // (row / 2) % 4 for 64-byte rows)
+    const int xr = D == 128 ? (r & 7) : ((r >> 1) & 3);
+    uint8_t* orow = out_tiles + (it & 1) * C::kOutBytes + r * D;
 #pragma unroll
-    for (int ps = 0; ps < PASSES; ++ps) {
-      const int r = ps * RPP + rip;
-      if (row0 + r < p.N) {
-        uint2 out;
-        out.x = quant4_e4m3(&y[ps][0], s, r_lo, r_hi, fast);
-        out.y = quant4_e4m3(&y[ps][4], s, r_lo, r_hi, fast);
-        *reinterpret_cast<uint2*>(out_blk + static_cast<size_t>(r) * D + seg * 8) = out;
-      }
+    for (int g = 0; g < 4; ++g) {
+      uint4 v;
+      v.x = quant4_e4m3(&y[16 * g], s, r_lo, r_hi, fast);
+      v.y = quant4_e4m3(&y[16 * g + 4], s, r_lo, r_hi, fast);
+      v.z = quant4_e4m3(&y[16 * g + 8], s, r_lo, r_hi, fast);
+      v.w = quant4_e4m3(&y[16 * g + 12], s, r_lo, r_hi, fast);
+      *reinterpret_cast<uint4*>(orow + (((hc * 4 + g) ^ xr) << 4)) = v;
+    }
+    fence_proxy_async_smem();   // generic writes, read next by the TMA store
+    __syncthreads();
+    if (tid == 0) {
+      const int bh = t / p.n_blocks;
+      tma_store_4d(&p.tm_x8, out_tiles + (it & 1) * C::kOutBytes, 0, row0, bh % p.H, bh / p.H);
+      bulk_commit_group();
     }
   }
+  if (tid == 0) bulk_wait_group<0>();   // the last stores have landed
 
   // After a wait gave up, let the copies still in flight land (bounded)
   // before the CTA's shared memory is released.

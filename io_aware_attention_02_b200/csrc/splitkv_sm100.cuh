@@ -1,4 +1,5 @@
-// Split-KV attention forward for sm_100a (bf16 / fp16, head dim 64 or 128):
+// Split-KV attention forward for sm_100a (bf16 / fp16, head dim 64, 128 or
+// 256):
 // short query blocks against long key/value sequences, the keys of each
 // (head, query tile) divided among CTAs and the partial results merged.
 //
@@ -23,7 +24,8 @@
 // is (b*h, 128-row query tile, split).  Warp 0 issues TMA loads (Q once per
 // unit, then K and V tiles in the order the MMA consumes them), warp 1 issues
 // tcgen05 products, warps 4-7 run the online softmax (thread = query row).
-// S is double-buffered in TMEM (S_a | S_b | O), so the product S(j+1) runs
+// S is double-buffered in TMEM (S_a | S_b | O: 128 + 128 + d <= 512
+// columns), so the product S(j+1) runs
 // while the softmax works on S(j); P is written over its S buffer and
 // O += P V_j reads it from TMEM.  Warps whose 32 rows are all past Nq skip the
 // arithmetic (decode tiles are mostly padding rows).  Each unit writes its
@@ -50,7 +52,9 @@ struct SplitCfg {
   static constexpr int kChunkBytes = 128 * 128;
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = (D == 64) ? 10 : 6;    // K/V ring (deep: the decode shapes stream from HBM)
+  // K/V ring (deep where it fits: the decode shapes stream from HBM); at
+  // d = 256 a tile is 64 KiB and only two fit beside Q
+  static constexpr int kStages = (D == 64) ? 10 : (D == 128 ? 6 : 2);
   static constexpr int kOffKV = kTileBytes;             // [Q | ring | barriers]
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kSmem = kOffBar + 512 + 1024;
@@ -302,6 +306,7 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
             for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(rr[i]);
           }
           tmem_wait_ld();
+          tmem_reg_fence(s);
           const int key0 = (j0 + jj) * 128;
           const bool need_mask = (CAUSAL && key0 + 127 > qt * 128 + p.q_off) || (key0 + 128 > p.Nk);
           if (need_mask) {
@@ -327,9 +332,12 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
               uint32_t rr[32];
               tmem_ld32(tO + cc * 32, rr);
               tmem_wait_ld();
+              tmem_reg_fence(rr);
 #pragma unroll
               for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
               tmem_st32(tO + cc * 32, rr);
+              tmem_wait_st();     // the store reads rr asynchronously
+              tmem_reg_fence(rr);
             }
           }
           // a row that has seen no visible key yet keeps m = -inf: its P is 0
@@ -362,6 +370,7 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
         uint32_t rr[32];
         tmem_ld32(tO + cc * 32, rr);
         tmem_wait_ld();
+        tmem_reg_fence(rr);
         if (row < p.Nq) {
 #pragma unroll
           for (int g4 = 0; g4 < 8; ++g4)
@@ -397,9 +406,9 @@ __global__ void __launch_bounds__(256) attn_splitkv_combine_kernel(const float* 
   for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, lse_part[(static_cast<size_t>(s) * BH + bh) * Nq + row]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // each lane owns 4 columns of every 128-column group (d_out <= 256)
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   float wsum = 0.f;
-  const int col = 4 * lane;
   if (mx != -INFINITY) {
     for (int s = 0; s < ns; ++s) {
       const size_t prow = (static_cast<size_t>(s) * BH + bh) * Nq + row;
@@ -407,22 +416,30 @@ __global__ void __launch_bounds__(256) attn_splitkv_combine_kernel(const float* 
       if (ls == -INFINITY) continue;
       const float wgt = __expf(ls - mx);
       wsum += wgt;
-      if (col < d_out) {
-        const float4 x = *reinterpret_cast<const float4*>(o_part + prow * d_out + col);
-        acc[0] = fmaf(wgt, x.x, acc[0]);
-        acc[1] = fmaf(wgt, x.y, acc[1]);
-        acc[2] = fmaf(wgt, x.z, acc[2]);
-        acc[3] = fmaf(wgt, x.w, acc[3]);
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int col = 128 * g + 4 * lane;
+        if (col < d_out) {
+          const float4 x = *reinterpret_cast<const float4*>(o_part + prow * d_out + col);
+          acc[g][0] = fmaf(wgt, x.x, acc[g][0]);
+          acc[g][1] = fmaf(wgt, x.y, acc[g][1]);
+          acc[g][2] = fmaf(wgt, x.z, acc[g][2]);
+          acc[g][3] = fmaf(wgt, x.w, acc[g][3]);
+        }
       }
     }
   }
   const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
   const size_t orow = static_cast<size_t>(bh) * Nq + row;
-  if (col < d_out) {
-    uint2 v;
-    v.x = pack2<T>(acc[0] * inv, acc[1] * inv);
-    v.y = pack2<T>(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(o + orow * d_out + col) = v;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int col = 128 * g + 4 * lane;
+    if (col < d_out) {
+      uint2 v;
+      v.x = pack2<T>(acc[g][0] * inv, acc[g][1] * inv);
+      v.y = pack2<T>(acc[g][2] * inv, acc[g][3] * inv);
+      *reinterpret_cast<uint2*>(o + orow * d_out + col) = v;
+    }
   }
   if (lse != nullptr && lane == 0) lse[orow] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
 }

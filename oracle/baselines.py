@@ -18,7 +18,10 @@ casts.  Readings where the page is silent: scores accumulate in fp32 from
 the rounded inputs; the softmax is computed in fp32 and its normalised
 result rounded to fp16; for FP8 the fp16 probabilities are rounded to e4m3
 with one per-tensor scale (448 / max P) before the P.V product, which
-accumulates in fp32; the output is rounded to fp16.
+accumulates in fp32; the output is rounded to fp16.  The fp16 baseline has a
+second reading of "intermediate results in FP16" (``round_scores=True``):
+the score matrix itself is also rounded to fp16 before the softmax, as an
+eager fp16 attention does when its Q.K^T product returns fp16.
 
 The ratios themselves are measured, not asserted by the pages' numbers:
 "parity unpinned" for the 1.7x / 2.6x values.
@@ -38,11 +41,14 @@ def _masked(s, causal):
     return s
 
 
-def standard_fp16_attention(q, k, v, scale, causal=False):
-    """FP16 standard attention of one head: fp16 inputs, fp32 scores,
-    softmax written out in fp16, fp32 accumulation of P.V, fp16 output."""
+def standard_fp16_attention(q, k, v, scale, causal=False, round_scores=False):
+    """FP16 standard attention of one head: fp16 inputs, fp32 scores (rounded
+    to fp16 when ``round_scores``), softmax written out in fp16, fp32
+    accumulation of P.V, fp16 output."""
     q16, k16, v16 = (np.asarray(x, dtype=np.float16) for x in (q, k, v))
     s = (q16.astype(np.float32) @ k16.astype(np.float32).T) * np.float32(scale)
+    if round_scores:
+        s = s.astype(np.float16).astype(np.float32)
     s = _masked(s, causal)
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m, dtype=np.float32)

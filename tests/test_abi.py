@@ -33,7 +33,9 @@ def test_header_declares_the_boundary():
                                   "attn_fwd_noalloc", "attn_fwd_strided", "attn_bwd",
                                   "attn_bwd_workspace_bytes", "attn_fwd_splitkv",
                                   "attn_fwd_splitkv_workspace_bytes", "attn_fwd_splitkv_auto_splits",
-                                  "attn_fwd_host", "attn_fwd_host_workspace_bytes"])
+                                  "attn_fwd_host", "attn_fwd_host_workspace_bytes",
+                                  "attn_noalloc_last_status", "attn_debug_status_allocated",
+                                  "attn_debug_set_ablation"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -91,7 +93,9 @@ def test_quant_and_fp8_validation(lib):
     args = [GOOD] * 8 + [1, 1, 128, 128, 0.1, 0, 0, None]
     bad = list(args); bad[3] = None
     assert F(*bad) == binding.ATTN_ERR_INVALID_ARG
-    bad = list(args); bad[11] = 64
+    bad = list(args); bad[11] = 96
+    assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
+    bad = list(args); bad[11] = 64; bad[14] = 1      # the V transposer needs 128-byte rows
     assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
     bad = list(args); bad[0] = GOOD + 1
     assert F(*bad) == binding.ATTN_ERR_MISALIGNED
@@ -174,7 +178,7 @@ def test_splitkv_validation(lib):
     assert call(causal=1, Nq=2000) == binding.ATTN_ERR_INVALID_ARG     # queries past the keys
     assert call(ns=-1) == binding.ATTN_ERR_INVALID_ARG
     assert call(scale=float("nan")) == binding.ATTN_ERR_INVALID_ARG
-    assert call(d=136) == binding.ATTN_ERR_UNSUPPORTED
+    assert call(d=264) == binding.ATTN_ERR_UNSUPPORTED
     assert call(d=100) == binding.ATTN_ERR_UNSUPPORTED
     assert call(dtype=5) == binding.ATTN_ERR_UNSUPPORTED
     assert call(o=GOOD + 8) == binding.ATTN_ERR_MISALIGNED
@@ -208,6 +212,8 @@ def test_host_forward_validation(lib):
 
 def test_debug_hook_validation(lib):
     assert lib.attn_debug_set_fault(5, 0) == binding.ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_set_ablation(2) == binding.ATTN_ERR_INVALID_ARG
+    assert lib.attn_debug_set_ablation(-1) == binding.ATTN_ERR_INVALID_ARG
     assert lib.attn_debug_set_fault(0, 0) == binding.ATTN_OK
 
 

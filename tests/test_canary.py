@@ -1,8 +1,7 @@
 """Canary checks of the outputs: every output buffer is filled with NaN (or
 the e4m3 NaN code) before the call, so an element a kernel forgets to write
 shows up, and an output view inside a larger NaN-filled buffer shows any
-write outside the view.  These stand in for an uninitialised-memory checker.
-Kept in a file that pytest collects last."""
+write outside the view.  These stand in for an uninitialised-memory checker."""
 
 import math
 

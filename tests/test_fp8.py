@@ -114,6 +114,32 @@ def test_fp8_attention_vs_fp64_oracle(lib, causal, hadamard, N):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hadamard", [False, True])
+@pytest.mark.parametrize("N", [1, 128, 300, 1500])
+def test_fp8_head_dim_64(lib, causal, hadamard, N):
+    """Head dim 64: 64-byte e4m3 rows (64-byte swizzle for TMA and the
+    tensor-core operands), same parity bars as d = 128 against the fp64
+    oracle on outlier inputs, and against exact attention on the
+    dequantised operands.  (At N = 1 the output is one row of V after e4m3
+    rounding, with nothing to average the rounding out: only the second
+    comparison applies there.)"""
+    q, k, v = _x(2, 3, N, 64, seed=40 + N)
+    signs = inputs.hadamard_signs(64, seed=2)
+    o, lse, packed = _fp8_attention(lib, q, k, v, causal, hadamard, signs)
+    assert lib.last_status()[0] == 0
+    scale = 1 / math.sqrt(64)
+    if N > 1:
+        o_ref, l_ref = A.attention(q, k, v, scale, causal)
+        err = errors(o.cpu(), lse.cpu(), o_ref, l_ref)
+        assert err["rmse"] <= FP8_RMSE, err
+    q8, k8, v8, qd, kd, vd = (t.cpu().numpy() for t in packed)
+    o_q, l_q = A.attention(F.dequantize_blocks(q8, qd), F.dequantize_blocks(k8, kd),
+                           F.dequantize_blocks(v8, vd), scale, causal)
+    err_q = errors(o.cpu(), lse.cpu(), o_q, l_q)
+    assert err_q["rmse"] <= 1.5e-2 and err_q["lse_max_abs"] <= 5e-3, err_q
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_fp8_headline_shape_sampled(lib, causal):
     """B=4, H=16, N=8192, d=128 with outliers; Hadamard on; sampled rows."""
     q, k, v = _x(4, 16, 8192, 128, seed=0)
@@ -155,7 +181,9 @@ def test_accuracy_vs_low_precision_baselines(lib):
     attention, and the fp16 kernel (fp32 statistics) more accurate than a
     standard fp16 attention that writes its softmax out in fp16.  The pages
     report 2.6x and 1.7x (baselines whose rounding they do not describe);
-    measured here 1.59x and 1.03x; only the direction is asserted."""
+    measured here 1.59x and, for the fp16 baseline, 1.03x when only its
+    softmax output is fp16 and more when its scores are rounded to fp16 as
+    well; only the direction is asserted."""
     from oracle import baselines as Bl
     N, d = 1024, 128
     scale = 1 / math.sqrt(d)
@@ -165,7 +193,7 @@ def test_accuracy_vs_low_precision_baselines(lib):
     q16, k16, v16 = (t.to(torch.float16) for t in (q, k, v))
     o16, _ = lib.fwd(q16.cuda(), k16.cuda(), v16.cuda(), scale=scale)
     torch.cuda.synchronize()
-    e8, e8b, e16, e16b = [], [], [], []
+    e8, e8b, e16, e16b, e16s = [], [], [], [], []
     for h in range(2):
         qq, kk, vv = (t[0, h].double().numpy() for t in (q, k, v))
         o_ref, _ = A.attention_head(qq, kk, vv, scale)
@@ -175,9 +203,12 @@ def test_accuracy_vs_low_precision_baselines(lib):
         o_ref16, _ = A.attention_head(q6, k6, v6, scale)
         e16.append(Bl.rmse(o16[0, h].double().cpu().numpy(), o_ref16))
         e16b.append(Bl.rmse(Bl.standard_fp16_attention(q6, k6, v6, scale), o_ref16))
+        e16s.append(Bl.rmse(Bl.standard_fp16_attention(q6, k6, v6, scale, round_scores=True), o_ref16))
     ratio8 = float(np.mean(e8b) / np.mean(e8))
     ratio16 = float(np.mean(e16b) / np.mean(e16))
+    ratio16s = float(np.mean(e16s) / np.mean(e16))
     print(f"RMSE ratios: per-tensor FP8 / ours {ratio8:.2f} (pages 2.6), standard fp16 / ours {ratio16:.2f} "
-          f"(pages 1.7)")
+          f"(fp16 softmax output), {ratio16s:.2f} (fp16 scores and softmax output) (pages 1.7)")
+    assert np.mean(e16) < np.mean(e16s), (e16, e16s)
     assert np.mean(e8) < np.mean(e8b), (e8, e8b)
     assert np.mean(e16) < np.mean(e16b), (e16, e16b)

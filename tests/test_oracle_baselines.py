@@ -24,6 +24,25 @@ def test_baselines_exact_on_representable_uniform_case():
     np.testing.assert_array_equal(Bl.per_tensor_fp8_attention(q, k, v, 0.5), o_ref)
 
 
+def test_fp16_score_rounding_reading():
+    """The second reading of the fp16 baseline differs from the first only by
+    rounding the scores to fp16: with scores that fp16 holds exactly (small
+    integers times a power-of-two scale) the two agree bit for bit; with
+    Gaussian scores they differ, and the extra rounding raises the error."""
+    rng = np.random.default_rng(3)
+    q = rng.integers(-3, 4, size=(64, 8)).astype(np.float64)
+    k = rng.integers(-3, 4, size=(64, 8)).astype(np.float64)
+    v = rng.standard_normal((64, 8))
+    for causal in (False, True):
+        np.testing.assert_array_equal(Bl.standard_fp16_attention(q, k, v, 0.25, causal),
+                                      Bl.standard_fp16_attention(q, k, v, 0.25, causal, round_scores=True))
+    x = [inputs.head_f32(2, t, 0, 0, 512, 64).astype(np.float64) for t in "qkv"]
+    o_ref, _ = A.attention_head(*x, 1 / 8)
+    e_a = Bl.rmse(Bl.standard_fp16_attention(*x, 1 / 8), o_ref)
+    e_b = Bl.rmse(Bl.standard_fp16_attention(*x, 1 / 8, round_scores=True), o_ref)
+    assert e_a < e_b < 5 * e_a + 1e-3, (e_a, e_b)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_baselines_close_but_not_exact_on_gaussian(causal):
     x = [inputs.head_f32(0, t, 0, 0, 256, 64).astype(np.float64) for t in "qkv"]

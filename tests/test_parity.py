@@ -221,3 +221,25 @@ def test_strided_padded_rows_and_mixed_layouts(lib):
     torch.cuda.synchronize()
     err = errors(o.cpu(), lse.cpu(), *A.attention(q, k, v, 1 / math.sqrt(d), False))
     assert_bf16_ok(err, "padded rows")
+
+
+@pytest.mark.parametrize("causal,N", [(False, 1000), (True, 777), (True, 2048)])
+def test_serialised_tile_schedule_is_bit_identical(lib, causal, N):
+    """The ablation switch (attn_debug_set_ablation) changes only the
+    schedule of the two query tiles, not the arithmetic: outputs are equal
+    bit for bit to the ping-pong schedule's.  Other head dims are refused
+    while it is on."""
+    q, k, v = (t.cuda() for t in inputs.qkv(1, 3, N, 128, seed=N))
+    o0, l0 = lib.fwd(q, k, v, causal=causal)
+    x64 = q[..., :64].contiguous()
+    try:
+        lib.debug_set_ablation(1)
+        o1, l1 = lib.fwd(q, k, v, causal=causal)
+        with pytest.raises(lib.AttnError) as e:
+            lib.fwd(x64, x64, x64)
+        assert e.value.code == lib.ATTN_ERR_UNSUPPORTED
+    finally:
+        lib.debug_set_ablation(0)
+    torch.cuda.synchronize()
+    assert lib.last_status()[0] == 0
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)

@@ -43,7 +43,7 @@ def _run(lib, B, H, Nq, Nk, d, causal, n_splits=0, seed=0, dtype=torch.bfloat16,
     return errors(o_g, l_g, o_ref, l_ref)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 128), (1, 129), (1, 4096), (7, 1000), (16, 3000), (128, 2048),
                                    (129, 700), (300, 300), (1, 20000)])
@@ -61,7 +61,7 @@ def test_split_counts(lib, n_splits, causal):
     assert_bf16_ok(err, (n_splits, causal))
 
 
-@pytest.mark.parametrize("d", [8, 40, 96, 120])
+@pytest.mark.parametrize("d", [8, 40, 96, 120, 136, 248])
 def test_head_dims_padded(lib, d):
     err = _run(lib, 1, 2, 3, 1500, d, True, seed=d)
     assert_bf16_ok(err, ("d", d))
@@ -110,7 +110,7 @@ def test_auto_split_count_covers_the_sms(lib):
 
 
 def test_bad_arguments_raise(lib):
-    q = torch.zeros(1, 1, 4, 256, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 1, 4, 264, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lib.AttnError):
         lib.fwd_splitkv(q, q, q)
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16, device="cuda")
