@@ -164,14 +164,18 @@ enum : int {
 // Softmax arithmetic helpers
 // ---------------------------------------------------------------------------
 
-// max of 128 values with 3-input max instructions, four independent chains.
+// max of 128 values with 3-input max instructions, four independent chains:
+// s[0..3] start the chains, 15 steps of 8 cover s[4..123], s[124..127] close
+// them (every index stays inside the array).
 __device__ __forceinline__ float row_max128(const float (&s)[128]) {
   float a[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-  for (int i = 4; i < 128; i += 8) {
+  for (int i = 4; i < 124; i += 8) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 4 + k]);
   }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], s[124 + k]);
   return fmax3(fmaxf(a[0], a[1]), a[2], a[3]);
 }
 

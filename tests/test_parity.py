@@ -243,3 +243,22 @@ def test_serialised_tile_schedule_is_bit_identical(lib, causal, N):
     torch.cuda.synchronize()
     assert lib.last_status()[0] == 0
     assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_key_with_negative_score_returns_v(lib, d, causal):
+    """N = 1: the only key gets P = 1, so O = V bit for bit and LSE = the
+    score, also when that score is negative and every other column of the
+    128-key tile is masked (the row max must see only the masked tile: a max
+    that also took in the masked columns' zero scores would lift m to 0,
+    round P = exp(s) < 1 to 16 bits and move O off V)."""
+    q = inputs.qkv(2, 3, 1, d, seed=d)[0]
+    k = -q                                          # <q, k> < 0 for every head
+    v = inputs.qkv(2, 3, 1, d, seed=d + 1)[2]
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = lib.fwd(qd, kd, vd, causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o, vd)
+    s = (q.double() * k.double()).sum(-1) / math.sqrt(d)
+    assert float((lse.double().cpu() - s).abs().max()) <= 1e-5 * max(1.0, float(s.abs().max()))
