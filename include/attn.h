@@ -114,7 +114,7 @@ attn_status_t attn_fwd_strided(const void* q, const void* k, const void* v, void
  *             (Sylvester H_d) before quantising.  Use it for Q and K only.
  *   signs   : d fp32 values of +-1 (device pointer), or NULL for all +1.
  *             Ignored when hadamard = 0.  Q and K must use the same signs.
- *   d       : 64 or 128.
+ *   d       : 64, 128 or 256 (others -> ATTN_ERR_UNSUPPORTED).
  * Per block: amax = max |y|; s = amax / 448 in fp32 (s = 1 if amax = 0);
  * code = e4m3_rn_satfinite(y / s) with an IEEE fp32 division.
  */
@@ -130,12 +130,12 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
  *                rotated).
  *   q_descale, k_descale, v_descale : [B][H][ceil(N/128)] fp32 factors.
  *   o   : [B][H][N][d] bf16, written.   lse : [B][H][N] fp32 or NULL.
- *   d   : 64 or 128 (others -> ATTN_ERR_UNSUPPORTED).
+ *   d   : 64, 128 or 256 (others -> ATTN_ERR_UNSUPPORTED).
  *   v_transpose : 0 = feed V to the tensor core MN-major, straight from the
  *                 TMA tile; 1 = transpose each V tile in shared memory to
  *                 K-major first (the pages' layout step; sm_100a accepts
  *                 either, both give identical results).  1 needs d = 128
- *                 (ATTN_ERR_UNSUPPORTED at d = 64).
+ *                 (ATTN_ERR_UNSUPPORTED at d = 64 and 256).
  * Scores use scale * q_descale * k_descale per (query block, key block);
  * P is rounded to e4m3 after multiplying by 256 * v_descale[j] / max_j
  * v_descale[j]; statistics are fp32 and l sums the unrounded P.

@@ -194,7 +194,7 @@ attn_status_t launch_fwd_c(const attn::FwdParams& p, int grid, int causal, cudaS
 // 128-row tiles).
 template <typename E, bool CAUSAL>
 attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream) {
-  using Cfg = attn::Fwd256Cfg;
+  using Cfg = attn::Fwd256Cfg<E>;
   auto kern = attn::attn_fwd_sm100_d256_kernel<E, CAUSAL>;
   static AttrFlags attr_done;
   if (attr_needed(attr_done)) {
@@ -206,7 +206,7 @@ attn_status_t launch_fwd256(attn::FwdParams p, int sm_count, cudaStream_t stream
   p.n_qpairs = (p.N + 127) / 128;
   p.n_units = p.BH * p.n_qpairs;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
-  set_schedule(&p, CAUSAL ? 1 : 0, p.n_qpairs, grid, kv_bytes_of(p.BH, p.N, 256, 2));
+  set_schedule(&p, CAUSAL ? 1 : 0, p.n_qpairs, grid, kv_bytes_of(p.BH, p.N, 256, Cfg::kBytes));
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -514,7 +514,7 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
     return ATTN_ERR_INVALID_ARG;
   if (hadamard != 0 && hadamard != 1) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(descale) & 3u) != 0 ||
       (signs != nullptr && (reinterpret_cast<uintptr_t>(signs) & 3u) != 0))
     return ATTN_ERR_MISALIGNED;
@@ -525,8 +525,11 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
   if ((r = make_map(&p.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, H, N, d, contiguous(H, N, d), 64)) !=
       ATTN_OK)
     return r;
-  // codes: one box spans a whole row of d bytes (64-byte swizzle at d = 64)
-  if ((r = make_map(&p.tm_x8, x8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, H, N, d, contiguous(H, N, d), d)) != ATTN_OK)
+  // codes: one box spans a row of d bytes (64-byte swizzle at d = 64), or
+  // half a row at d = 256
+  const int box8 = d < 128 ? d : 128;
+  if ((r = make_map(&p.tm_x8, x8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, H, N, d, contiguous(H, N, d), box8)) !=
+      ATTN_OK)
     return r;
   p.descale = descale;
   p.signs = signs;
@@ -538,6 +541,7 @@ attn_status_t attn_quant_fp8(const void* x, void* x8, float* descale, int B, int
   p.total = p.n_blocks * B * H;
   p.hadamard = hadamard;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256) return launch_quant<256>(p, st->sm_count, s);
   return d == 64 ? launch_quant<64>(p, st->sm_count, s) : launch_quant<128>(p, st->sm_count, s);
 }
 
@@ -552,7 +556,7 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   if (r != ATTN_OK) return r;
   if (v_transpose != 0 && v_transpose != 1) return ATTN_ERR_INVALID_ARG;
   if (d < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   if (v_transpose && d != 128) return ATTN_ERR_UNSUPPORTED;   // the transposer handles 128-byte rows
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
   const uintptr_t a4 = reinterpret_cast<uintptr_t>(q_descale) | reinterpret_cast<uintptr_t>(k_descale) |
@@ -566,10 +570,12 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   attn::FwdParams p{};
   const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const Strides c8 = contiguous(H, N, d);
-  // one box spans a whole e4m3 row: 128 bytes (64-byte swizzle at d = 64)
-  if ((r = make_map(&p.tm_q, q8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_k, k8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
-  if ((r = make_map(&p.tm_v, v8, dt, 1, B, H, N, d, c8, d)) != ATTN_OK) return r;
+  // one box spans a whole e4m3 row of 128 bytes (64-byte swizzle at d = 64),
+  // or half a row at d = 256
+  const int box = d < 128 ? d : 128;
+  if ((r = make_map(&p.tm_q, q8, dt, 1, B, H, N, d, c8, box)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_k, k8, dt, 1, B, H, N, d, c8, box)) != ATTN_OK) return r;
+  if ((r = make_map(&p.tm_v, v8, dt, 1, B, H, N, d, c8, box)) != ATTN_OK) return r;
   p.q_desc = q_descale;
   p.k_desc = k_descale;
   p.v_desc = v_descale;
@@ -581,6 +587,9 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const
   const int grid = p.n_units < st->sm_count ? p.n_units : st->sm_count;
   set_schedule(&p, causal, p.n_qpairs, grid, kv_bytes_of(BH, N, d, 1));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256)
+    return causal ? launch_fwd256<__nv_fp8_e4m3, true>(p, st->sm_count, s)
+                  : launch_fwd256<__nv_fp8_e4m3, false>(p, st->sm_count, s);
   if (v_transpose)
     return causal ? launch_fwd<__nv_fp8_e4m3, 128, true, true>(p, grid, s)
                   : launch_fwd<__nv_fp8_e4m3, 128, false, true>(p, grid, s);

@@ -1,4 +1,5 @@
-// Fused attention forward for sm_100a, head dim 256 (bf16 / fp16).
+// Fused attention forward for sm_100a, head dim 256 (bf16 / fp16, and e4m3
+// with per-block descale factors as in fwd_sm100.cuh).
 //
 // Same computation as fwd_sm100.cuh (exact attention with online softmax,
 // running max m and sum l, division by l at the end; droidorbit.com,
@@ -15,19 +16,24 @@
 //
 // Roles (256 threads): warp 0 TMA, warp 1 MMA issuer (one thread) and TMEM
 // allocator, warps 4-7 softmax (one thread per query row).  Shared memory:
-// Q (64 KiB) and a two-stage K/V ring of 64 KiB tiles.  P of key tile j is
-// written over S(j) as 16-bit pairs and published in two 64-key halves.
-// Before publishing P(j) the softmax waits for PV(j-1) (it may rescale O).
+// Q (64 KiB) and a two-stage K/V ring of 64 KiB tiles (e4m3: 32 KiB tiles, a
+// four-stage ring).  P of key tile j is written over S(j) as 16-bit pairs (or
+// e4m3 quads) and published in two 64-key halves.  Before publishing P(j)
+// the softmax waits for PV(j-1) (it may rescale O).
 #pragma once
 #include "fwd_sm100.cuh"
 
 namespace attn {
 
+template <typename E>
 struct Fwd256Cfg {
-  static constexpr int kChunkBytes = 128 * 128;   // 128 rows x 128 bytes (64 columns)
-  static constexpr int kChunks = 4;               // 256 columns
-  static constexpr int kTileBytes = kChunks * kChunkBytes;   // 64 KiB
-  static constexpr int kStages = 2;
+  static constexpr int kBytes = Elem<E>::kBytes;
+  static constexpr int kChunkBytes = 128 * 128;   // 128 rows x 128 bytes
+  static constexpr int kChunkCols = 128 / kBytes; // columns per chunk
+  static constexpr int kChunks = 256 / kChunkCols;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;   // 64 KiB (32 KiB e4m3)
+  static constexpr int kStages = kBytes == 2 ? 2 : 4;
+  static constexpr int kKeysPerMma = 32 / kBytes; // 32 bytes of K per tcgen05.mma
   static constexpr int kThreads = 256;
   static constexpr int kTmemCols = 512;           // S_a | S_b | O
   static constexpr int kColO = 256;
@@ -48,8 +54,9 @@ __device__ __forceinline__ uint32_t seq_v(int j, int n) {
 
 template <typename E, bool CAUSAL>
 __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __grid_constant__ FwdParams p) {
-  using Cfg = Fwd256Cfg;
+  using Cfg = Fwd256Cfg<E>;
   using T = typename Elem<E>::Out;
+  constexpr bool kF8 = Elem<E>::kF8;
   constexpr int D = 256;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -120,7 +127,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * 64, qt * 128, bh % p.H, bh / p.H);
+          tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * Cfg::kChunkCols, qt * 128, bh % p.H,
+                      bh / p.H);
         for (int q = 0; q < 2 * n && ok; ++q, ++kv_iter) {
           // q -> (K or V, key tile j), inverse of seq_k / seq_v
           const bool is_v = (q == 2 * n - 1) || (q > 0 && (q & 1) == 0);
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
           const CUtensorMap* map = is_v ? &p.tm_v : &p.tm_k;
           for (int c = 0; c < Cfg::kChunks; ++c)
             tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
-                        c * 64, j * 128, bh % p.H, bh / p.H);
+                        c * Cfg::kChunkCols, j * 128, bh % p.H, bh / p.H);
         }
       }
       if (!ok) {
@@ -163,21 +171,25 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       auto issue_s = [&](int buf, uint32_t kstage) {
         const uint64_t b0 = dK + static_cast<uint64_t>((kstage * Cfg::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
+          // 32 bytes of the head dim per product, four per 128-byte chunk row
           const uint32_t off = ((kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + buf * 128, dQ + off, b0 + off, idesc_s, kk > 0, false);
+          mma_ss(tmem + buf * 128, dQ + off, b0 + off, idesc_s, kk > 0, kF8);
         }
       };
-      // O += P(j) V_j, each 64-key half as soon as it is published.
+      // O += P(j) V_j, each 64-key half as soon as it is published.  P:
+      // kKeysPerMma keys = 8 TMEM columns per product; V: MN-major,
+      // kKeysPerMma rows of 128-byte chunks per product.
       auto pv = [&](int buf, uint32_t vstage, bool acc) -> bool {
         const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);
+        constexpr int kSteps = 64 / Cfg::kKeysPerMma;
         for (int h = 0; h < 2; ++h) {
           if (!mbar_wait(p_full + h, p_cnt & 1, p.status, abort_flag, kWherePFull, lim)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-            mma_ts(tmem + Cfg::kColO, tmem + buf * 128 + kk * 8, b0 + ((kk * 16 * 128) >> 4), idesc_o,
-                   (acc || kk > 0) ? 1u : 0u, false);
+          for (int kk = kSteps * h; kk < kSteps * (h + 1); ++kk)
+            mma_ts(tmem + Cfg::kColO, tmem + buf * 128 + kk * 8, b0 + ((kk * Cfg::kKeysPerMma * 128) >> 4),
+                   idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
         }
         ++p_cnt;
         return true;
@@ -241,7 +253,11 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
     const uint32_t tO = tmem + lane_off + Cfg::kColO;
     uint32_t s_cnt[2] = {0, 0}, or_cnt = 0, o_cnt = 0;
     bool ok = true;
-    constexpr float kLazy = 8.0f;
+    // e4m3: P is multiplied by a power-of-two gain times v_descale[j] / max
+    // v_descale before rounding, and the max may lag the true max by at most
+    // kLazy (log2 units), so that P * gain <= 256 * 2^0.75 < 448 stays finite
+    constexpr float kPGain = 256.0f;
+    constexpr float kLazy = kF8 ? 0.75f : 8.0f;
 
     for (int k = 0; ok; ++k) {
       const int unit = sched_unit(k, p.snake);
@@ -250,7 +266,17 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       decode_unit<CAUSAL>(unit, n_qt, p.BH, p.order, bh, qt);
       const int n = CAUSAL ? min(qt + 1, n_kv) : n_kv;
       const int row = qt * 128 + row_in_tile;
-      const float c = p.scale_log2;
+      float cq = p.scale_log2;   // score -> log2 domain factor (times the q descale for e4m3)
+      float vmax = 1.0f;         // e4m3: max v descale of this head
+      if constexpr (kF8) {
+        const size_t dbase = static_cast<size_t>(bh) * n_kv;
+        cq *= p.q_desc[dbase + min(qt, n_kv - 1)];
+        float vm = 0.f;
+        for (int b = lane; b < n_kv; b += 32) vm = fmaxf(vm, p.v_desc[dbase + b]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+        vmax = vm;
+      }
       float m = -INFINITY, l = 0.f;
 
       for (int j = 0; j < n; ++j) {
@@ -260,6 +286,13 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         ++s_cnt[buf];
         if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
+        float c = cq;
+        float pgain = 1.0f;
+        if constexpr (kF8) {
+          const size_t dbase = static_cast<size_t>(bh) * n_kv;
+          c = cq * p.k_desc[dbase + j];
+          pgain = kPGain * __fdiv_rn(p.v_desc[dbase + j], vmax);
+        }
 
         float s[128];
 #pragma unroll
@@ -287,22 +320,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         }
         // first half of P into registers, then (after PV(j-1) has finished)
         // the optional rescale of O and the publication of both halves
-        uint32_t pk0[32];
-        float sum;
-        {
-          const float2 c2 = make_float2(c, c);
-          const float2 nm2 = make_float2(-m, -m);
-          float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), c2, nm2);
-            const float2 pr = exp2_mufu2(x);
-            acc[i & 1] = __fadd2_rn(acc[i & 1], pr);
-            pk0[i] = pack2<T>(pr.x, pr.y);
-          }
-          const float2 a = __fadd2_rn(acc[0], acc[1]);
-          sum = a.x + a.y;
-        }
+        uint32_t pk0[kF8 ? 16 : 32];
+        float sum = exp_half<kF8, T, false>(s, 0, c, -m, pgain, pk0);
         if (j > 0) {
           w = mbar_wait(o_ready, or_cnt & 1, p.status, abort_flag, kWhereOFull, lim);
           ++or_cnt;
@@ -323,13 +342,11 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
             }
           }
         }
-        tmem_st32(tS, pk0);
-        tmem_wait_st();
-        tmem_reg_fence(pk0);
+        store_p_half<kF8>(tS, 0, pk0);
         tc_fence_before();
         mbar_arrive(p_full + 0);
-        sum += need_mask ? exp_pack_half<false, T, false>(s, 1, c, -m, 1.0f, tS)
-                         : exp_pack_half<false, T, true>(s, 1, c, -m, 1.0f, tS);
+        sum += need_mask ? exp_pack_half<kF8, T, false>(s, 1, c, -m, pgain, tS)
+                         : exp_pack_half<kF8, T, true>(s, 1, c, -m, pgain, tS);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + 1);
@@ -346,7 +363,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       ++o_cnt;
       if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; break; }
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = kF8 ? __fdiv_rn(vmax, kPGain * l) : 1.0f / l;
       // O rows are d_out wide (d_out <= D: smaller head dims run zero-padded
       // to D; the padding columns of O are zero and are not stored); O may be
       // strided over (batch, head, row)

@@ -217,20 +217,16 @@ __device__ __forceinline__ float2 exp2_mufu2(float2 x) {
 // Pairs i with (i % 8) < kPolyPairsPer8 take the polynomial path.
 constexpr int kPolyPairsPer8 = 1;
 
-// P = 2^(s*c - m) for one half (64 keys, h = 0 or 1) of a 128-key row:
-// packed to 16-bit pairs (or e4m3 quads, after the gain) and written over the
-// row's S columns in TMEM (32 columns per half at 16 bit, 16 at e4m3).  The
-// store has completed when it returns (tcgen05.st reads its source registers
-// asynchronously: they must not be reused before tcgen05.wait::st).
-// Returns the fp32 sum of the unrounded P of that half.
+// P = 2^(s*c - m) for one half (64 keys, h = 0 or 1) of a 128-key row,
+// packed to 16-bit pairs (or e4m3 quads, after the gain) into pk.  Returns the
+// fp32 sum of the unrounded P of that half.
 template <bool kF8, typename T, bool kPoly>
-__device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, float c, float neg_m,
-                                               float pgain, uint32_t tS) {
+__device__ __forceinline__ float exp_half(const float (&s)[128], int h, float c, float neg_m, float pgain,
+                                          uint32_t (&pk)[kF8 ? 16 : 32]) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(neg_m, neg_m);
   float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   if constexpr (!kF8) {
-    uint32_t pk[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int e = 64 * h + 2 * i;
@@ -239,12 +235,8 @@ __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, flo
       acc[i & 1] = __fadd2_rn(acc[i & 1], pr);
       pk[i] = pack2<T>(pr.x, pr.y);
     }
-    tmem_st32(tS + 32 * h, pk);
-    tmem_wait_st();
-    tmem_reg_fence(pk);
   } else {
     const float2 g2 = make_float2(pgain, pgain);
-    uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int e = 64 * h + 4 * i;
@@ -258,12 +250,34 @@ __device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, flo
       const float2 g1 = __fmul2_rn(p1, g2);
       pk[i] = pack4_e4m3(g0.x, g0.y, g1.x, g1.y);
     }
-    tmem_st16(tS + 16 * h, pk);
-    tmem_wait_st();
-    tmem_reg_fence(pk);
   }
   const float2 a = __fadd2_rn(acc[0], acc[1]);
   return a.x + a.y;
+}
+
+// Write one half of P over the row's S columns in TMEM (32 columns per half at
+// 16 bit, 16 at e4m3).  The store has completed when it returns: tcgen05.st
+// reads its source registers asynchronously, so they must not be reused
+// before tcgen05.wait::st.
+template <bool kF8>
+__device__ __forceinline__ void store_p_half(uint32_t tS, int h, uint32_t (&pk)[kF8 ? 16 : 32]) {
+  if constexpr (!kF8) {
+    tmem_st32(tS + 32 * h, pk);
+  } else {
+    tmem_st16(tS + 16 * h, pk);
+  }
+  tmem_wait_st();
+  tmem_reg_fence(pk);
+}
+
+// exp_half followed by store_p_half; returns the half's sum.
+template <bool kF8, typename T, bool kPoly>
+__device__ __forceinline__ float exp_pack_half(const float (&s)[128], int h, float c, float neg_m,
+                                               float pgain, uint32_t tS) {
+  uint32_t pk[kF8 ? 16 : 32];
+  const float sum = exp_half<kF8, T, kPoly>(s, h, c, neg_m, pgain, pk);
+  store_p_half<kF8>(tS, h, pk);
+  return sum;
 }
 
 // In-shared-memory transpose of one FP8 V tile (128 keys x 128 head-dim

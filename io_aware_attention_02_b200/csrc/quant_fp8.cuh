@@ -9,17 +9,19 @@
 // item 3.  The rotation leaves Q K^T unchanged because it is orthogonal.
 //
 // Streaming kernel: 2 bytes read and 1 byte written per element, meant to run
-// at HBM bandwidth.  Persistent CTAs of 128 * D/64 threads (two or three per
-// SM) walk the blocks of 128 rows of one (batch, head) in a strided order.
+// at HBM bandwidth.  Persistent CTAs of 128 * D/64 threads (three per SM at
+// D = 64, two at 128, one at 256) walk the blocks of 128 rows of one (batch,
+// head) in a strided order.
 // Thread 0 keeps a ring of kStages blocks in flight: each block arrives by
 // TMA (tile loads of 64 columns x 128 rows, 128-byte swizzle, rows past N
-// zero-filled).  A thread owns 64 columns of one row (the two threads of a
-// d = 128 row are neighbouring lanes): it reads them from shared memory (the
+// zero-filled).  A thread owns 64 columns of one row (the D/64 threads of a
+// row are neighbouring lanes): it reads them from shared memory (the
 // swizzle spreads a warp's 16-byte reads over all banks), applies the signs
 // (a flip of the bf16 sign bits), runs the six butterfly stages of the fast
 // Walsh-Hadamard transform that stay inside its 64 values in registers and,
-// at d = 128, the last stage with its neighbour by one lane shuffle per
-// value; then it scales by 1/sqrt(D) and takes its amax.  The block's amax
+// at d = 128 and 256, the remaining stages with its neighbours by one lane
+// shuffle per value and stage; then it scales by 1/sqrt(D) and takes its
+// amax.  The block's amax
 // needs every row, so the CTA meets at one barrier per block; that barrier
 // also tells thread 0 that the block's buffer has been read and may be
 // refilled.  Each thread then rounds its 64 values to e4m3 into one of two
@@ -35,7 +37,7 @@ enum : int { kWhereQuantFull = 10 };
 
 struct QuantParams {
   CUtensorMap tm_x;         // 4-D map over x (D, N, H, B): box 64 x 128, 128-byte swizzle
-  CUtensorMap tm_x8;        // 4-D map over the codes (D, N, H, B): box D x 128, D-byte swizzle
+  CUtensorMap tm_x8;        // 4-D map over the codes (D, N, H, B): box min(D, 128) x 128, same swizzle width
   float* descale;           // [BH][n_blocks]
   const float* signs;       // [D] or nullptr
   int* status;
@@ -51,10 +53,15 @@ struct QuantCfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   // input ring + two output staging tiles: 2 x 32 + 2 x 16 KiB per CTA and
-  // two CTAs per SM at D = 128; 3 x 16 + 2 x 8 KiB and three CTAs at D = 64
+  // two CTAs per SM at D = 128; 3 x 16 + 2 x 8 KiB and three CTAs at D = 64;
+  // 2 x 64 + 2 x 32 KiB and one CTA at D = 256
   static constexpr int kStages = D == 64 ? 3 : 2;
-  static constexpr int kMinBlocks = D == 64 ? 3 : 2;
+  static constexpr int kMinBlocks = D == 64 ? 3 : (D == 128 ? 2 : 1);
   static constexpr int kOutBytes = kRows * D;                // one block of codes
+  // the codes of a block go out in column chunks of at most 128 bytes (the
+  // widest swizzled box): one chunk up to D = 128, two at D = 256
+  static constexpr int kOutChunkCols = D < 128 ? D : 128;
+  static constexpr int kOutChunks = D / kOutChunkCols;
   static constexpr int kTpr = D / 64;                        // threads per row
   static constexpr int kThreads = 128 * kTpr;
   static constexpr int kWarps = kThreads / 32;
@@ -64,6 +71,7 @@ struct QuantCfg {
   static constexpr int kRedOff = kBarOff + 128;             // float [2][kWarps <= 8]
   static constexpr int kSgnOff = kBarOff + 256;             // uint32 [D / 2]: sign bits per bf16 pair
   static_assert(2 * kWarps * 4 <= 128, "amax slots overflow their region");
+  static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
   static constexpr int kSmem = kSgnOff + 2 * D + 1024;      // + alignment slack for the swizzle
   static_assert(kStages * 8 <= 64, "barriers overflow their slot");
 };
@@ -77,15 +85,18 @@ struct QuantCfg {
 // both ends of the bracket give the same code the quotient gives it too.
 // Otherwise the quotient lies within about 2^-20 of an e4m3 rounding
 // midpoint (a few values in ten thousand) and is taken by division.
-__device__ __forceinline__ uint32_t quant4_e4m3(const float* y, float s, float r_lo, float r_hi, bool fast) {
+// The four values come as two pairs; the products are taken two at a time
+// (each lane of a paired multiply rounds like the scalar one).
+__device__ __forceinline__ uint32_t quant4_e4m3(float2 y01, float2 y23, float s, float2 r_lo, float2 r_hi,
+                                                bool fast) {
   if (fast) {
-    const uint32_t a = pack4_e4m3(__fmul_rn(y[0], r_lo), __fmul_rn(y[1], r_lo), __fmul_rn(y[2], r_lo),
-                                  __fmul_rn(y[3], r_lo));
-    const uint32_t b = pack4_e4m3(__fmul_rn(y[0], r_hi), __fmul_rn(y[1], r_hi), __fmul_rn(y[2], r_hi),
-                                  __fmul_rn(y[3], r_hi));
+    const float2 a01 = __fmul2_rn(y01, r_lo), a23 = __fmul2_rn(y23, r_lo);
+    const float2 b01 = __fmul2_rn(y01, r_hi), b23 = __fmul2_rn(y23, r_hi);
+    const uint32_t a = pack4_e4m3(a01.x, a01.y, a23.x, a23.y);
+    const uint32_t b = pack4_e4m3(b01.x, b01.y, b23.x, b23.y);
     if (a == b) return a;
   }
-  return pack4_e4m3(__fdiv_rn(y[0], s), __fdiv_rn(y[1], s), __fdiv_rn(y[2], s), __fdiv_rn(y[3], s));
+  return pack4_e4m3(__fdiv_rn(y01.x, s), __fdiv_rn(y01.y, s), __fdiv_rn(y23.x, s), __fdiv_rn(y23.y, s));
 }
 
 template <int D>
@@ -153,8 +164,9 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
     const int row0 = (t % p.n_blocks) * C::kRows;
 
     // this thread's 64 values from the swizzled tile (16-byte piece q of the
-    // 64-column chunk sits at piece q ^ (row % 8) of the row's 128 bytes)
-    float y[64];
+    // 64-column chunk sits at piece q ^ (row % 8) of the row's 128 bytes),
+    // held as 32 pairs y[i] = (value 2i, value 2i + 1)
+    float2 y[32];
     const uint8_t* tile = smem + stage * C::kTileBytes + hc * C::kChunkBytes + r * 128;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -164,44 +176,55 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
         const uint4 m = reinterpret_cast<const uint4*>(sgn)[hc * 8 + q];
         raw.x ^= m.x; raw.y ^= m.y; raw.z ^= m.z; raw.w ^= m.w;
       }
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = unpack2<__nv_bfloat16>(w[i]);
-        y[q * 8 + 2 * i] = f.x;
-        y[q * 8 + 2 * i + 1] = f.y;
-      }
+      y[q * 4 + 0] = unpack2<__nv_bfloat16>(raw.x);
+      y[q * 4 + 1] = unpack2<__nv_bfloat16>(raw.y);
+      y[q * 4 + 2] = unpack2<__nv_bfloat16>(raw.z);
+      y[q * 4 + 3] = unpack2<__nv_bfloat16>(raw.w);
     }
     if (rot) {
-      // fast Walsh-Hadamard transform, one rounding per output of each stage:
-      // the stages over the 6 low index bits inside this thread ...
+      // fast Walsh-Hadamard transform, one rounding per output of each stage
+      // (index bit 0 first): bit 0 pairs the two values of a pair ...
 #pragma unroll
-      for (int h = 1; h < 64; h <<= 1) {
+      for (int i = 0; i < 32; ++i) {
+        const float a = y[i].x, b = y[i].y;
+        y[i] = make_float2(a + b, a - b);
+      }
+      // ... bits 1 to 5 pair whole pairs: one paired add and one paired
+      // multiply-add by -1 (an exact negation, then the one rounding of
+      // a - b) per two butterflies ...
+      const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
           if ((i & h) == 0) {
-            const float a = y[i], b = y[i | h];
-            y[i] = a + b;
-            y[i | h] = a - b;
+            const float2 a = y[i], b = y[i | h];
+            y[i] = __fadd2_rn(a, b);
+            y[i | h] = __ffma2_rn(b, neg1, a);
           }
         }
       }
-      // ... and at d = 128 the stage over index bit 6 with the neighbouring
-      // lane (lower chunk: y + other; upper chunk: other - y)
-      if constexpr (C::kTpr == 2) {
-        const float sg = hc == 0 ? 1.f : -1.f;
+      // ... and the index bits above 5 (bit 6 + s is bit s of the chunk
+      // index hc) with the lane that differs in that bit (lower chunk:
+      // y + other; upper chunk: other - y)
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float other = __shfl_xor_sync(0xffffffffu, y[i], 1);
-          y[i] = fmaf(sg, y[i], other);
+      for (int sb = 1; sb < C::kTpr; sb <<= 1) {
+        const float sg = (hc & sb) == 0 ? 1.f : -1.f;
+        const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 other = make_float2(__shfl_xor_sync(0xffffffffu, y[i].x, sb),
+                                           __shfl_xor_sync(0xffffffffu, y[i].y, sb));
+          y[i] = __ffma2_rn(sg2, y[i], other);
         }
       }
+      const float2 norm2 = make_float2(norm, norm);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) y[i] *= norm;
+      for (int i = 0; i < 32; ++i) y[i] = __fmul2_rn(y[i], norm2);
     }
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 64; i += 2) amax = fmax3(amax, fabsf(y[i]), fabsf(y[i + 1]));
+    for (int i = 0; i < 32; ++i) amax = fmax3(amax, fabsf(y[i].x), fabsf(y[i].y));
 
     // Block amax.  The slots alternate between blocks: a warp writes slot
     // set (it & 1) again only two barriers later, after every warp has read it.
@@ -235,27 +258,35 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
     const bool fast = s >= 0x1p-100f && s <= 0x1p100f;
     const float rc = __frcp_rn(s);
     const float r_lo = __fmul_rn(rc, 1.f - 0x1p-20f), r_hi = __fmul_rn(rc, 1.f + 0x1p-20f);
+    const float2 r_lo2 = make_float2(r_lo, r_lo), r_hi2 = make_float2(r_hi, r_hi);
 
-    // this thread's 64 codes: 16-byte pieces hc*4 + g of the row, swizzled
-    // the way the TMA store reads them (the D-byte swizzle XORs the 16-byte
-    // piece index with address bits 7 and up: row % 8 for 128-byte rows,
-    // (row / 2) % 4 for 64-byte rows)
-    const int xr = D == 128 ? (r & 7) : ((r >> 1) & 3);
-    uint8_t* orow = out_tiles + (it & 1) * C::kOutBytes + r * D;
+    // this thread's 64 codes: 16-byte pieces hc*4 + g of the row, in column
+    // chunk (hc*64) / kOutChunkCols, swizzled the way the TMA store reads
+    // them (the swizzle XORs the 16-byte piece index within the chunk row
+    // with address bits 7 and up: row % 8 for 128-byte rows, (row / 2) % 4
+    // for 64-byte rows)
+    const int xr = D >= 128 ? (r & 7) : ((r >> 1) & 3);
+    constexpr int kPiecesPerChunkRow = C::kOutChunkCols / 16;
+    const int piece0 = (hc * 4) % kPiecesPerChunkRow;
+    uint8_t* orow = out_tiles + (it & 1) * C::kOutBytes + ((hc * 4) / kPiecesPerChunkRow) * (C::kRows * C::kOutChunkCols) +
+                    r * C::kOutChunkCols;
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       uint4 v;
-      v.x = quant4_e4m3(&y[16 * g], s, r_lo, r_hi, fast);
-      v.y = quant4_e4m3(&y[16 * g + 4], s, r_lo, r_hi, fast);
-      v.z = quant4_e4m3(&y[16 * g + 8], s, r_lo, r_hi, fast);
-      v.w = quant4_e4m3(&y[16 * g + 12], s, r_lo, r_hi, fast);
-      *reinterpret_cast<uint4*>(orow + (((hc * 4 + g) ^ xr) << 4)) = v;
+      v.x = quant4_e4m3(y[8 * g], y[8 * g + 1], s, r_lo2, r_hi2, fast);
+      v.y = quant4_e4m3(y[8 * g + 2], y[8 * g + 3], s, r_lo2, r_hi2, fast);
+      v.z = quant4_e4m3(y[8 * g + 4], y[8 * g + 5], s, r_lo2, r_hi2, fast);
+      v.w = quant4_e4m3(y[8 * g + 6], y[8 * g + 7], s, r_lo2, r_hi2, fast);
+      *reinterpret_cast<uint4*>(orow + (((piece0 + g) ^ xr) << 4)) = v;
     }
     fence_proxy_async_smem();   // generic writes, read next by the TMA store
     __syncthreads();
     if (tid == 0) {
       const int bh = t / p.n_blocks;
-      tma_store_4d(&p.tm_x8, out_tiles + (it & 1) * C::kOutBytes, 0, row0, bh % p.H, bh / p.H);
+#pragma unroll
+      for (int c = 0; c < C::kOutChunks; ++c)
+        tma_store_4d(&p.tm_x8, out_tiles + (it & 1) * C::kOutBytes + c * (C::kRows * C::kOutChunkCols),
+                     c * C::kOutChunkCols, row0, bh % p.H, bh / p.H);
       bulk_commit_group();
     }
   }

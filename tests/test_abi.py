@@ -88,6 +88,7 @@ def test_quant_and_fp8_validation(lib):
     assert Q(None, GOOD, GOOD, 1, 1, 128, 128, 0, None, None) == binding.ATTN_ERR_INVALID_ARG
     assert Q(GOOD, GOOD, GOOD, 1, 1, 128, 128, 2, None, None) == binding.ATTN_ERR_INVALID_ARG
     assert Q(GOOD, GOOD, GOOD, 1, 1, 128, 96, 0, None, None) == binding.ATTN_ERR_UNSUPPORTED
+    assert Q(GOOD, GOOD, GOOD, 1, 1, 128, 512, 0, None, None) == binding.ATTN_ERR_UNSUPPORTED
     assert Q(GOOD + 4, GOOD, GOOD, 1, 1, 128, 128, 0, None, None) == binding.ATTN_ERR_MISALIGNED
     F = lib.attn_fwd_fp8
     args = [GOOD] * 8 + [1, 1, 128, 128, 0.1, 0, 0, None]
@@ -96,6 +97,10 @@ def test_quant_and_fp8_validation(lib):
     bad = list(args); bad[11] = 96
     assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
     bad = list(args); bad[11] = 64; bad[14] = 1      # the V transposer needs 128-byte rows
+    assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
+    bad = list(args); bad[11] = 256; bad[14] = 1
+    assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
+    bad = list(args); bad[11] = 512
     assert F(*bad) == binding.ATTN_ERR_UNSUPPORTED
     bad = list(args); bad[0] = GOOD + 1
     assert F(*bad) == binding.ATTN_ERR_MISALIGNED

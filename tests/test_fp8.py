@@ -20,7 +20,7 @@ def _x(B, H, N, d, seed, outliers=True):
     return inputs.qkv(B, H, N, d, seed=seed, outliers=outliers)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("N", [128, 300, 1024])
 def test_quant_plain_bit_exact(lib, d, N):
     x = _x(2, 3, N, d, seed=N)[0]
@@ -31,7 +31,7 @@ def test_quant_plain_bit_exact(lib, d, N):
     np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("signed", [False, True])
 def test_quant_hadamard_close(lib, d, signed):
     """With rotation the kernel's fp32 butterflies round differently from the
@@ -128,6 +128,30 @@ def test_fp8_head_dim_64(lib, causal, hadamard, N):
     o, lse, packed = _fp8_attention(lib, q, k, v, causal, hadamard, signs)
     assert lib.last_status()[0] == 0
     scale = 1 / math.sqrt(64)
+    if N > 1:
+        o_ref, l_ref = A.attention(q, k, v, scale, causal)
+        err = errors(o.cpu(), lse.cpu(), o_ref, l_ref)
+        assert err["rmse"] <= FP8_RMSE, err
+    q8, k8, v8, qd, kd, vd = (t.cpu().numpy() for t in packed)
+    o_q, l_q = A.attention(F.dequantize_blocks(q8, qd), F.dequantize_blocks(k8, kd),
+                           F.dequantize_blocks(v8, vd), scale, causal)
+    err_q = errors(o.cpu(), lse.cpu(), o_q, l_q)
+    assert err_q["rmse"] <= 1.5e-2 and err_q["lse_max_abs"] <= 5e-3, err_q
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("hadamard", [False, True])
+@pytest.mark.parametrize("N", [1, 128, 300, 1500])
+def test_fp8_head_dim_256(lib, causal, hadamard, N):
+    """Head dim 256: the one-tile kernel with S double-buffered in TMEM, its
+    e4m3 rows loaded as two 128-byte chunks; the rotation's last two
+    butterfly stages cross lanes in the quantiser.  Same bars as d = 64 and
+    128 (only the dequantised comparison at N = 1, as there)."""
+    q, k, v = _x(2, 3, N, 256, seed=50 + N)
+    signs = inputs.hadamard_signs(256, seed=5)
+    o, lse, packed = _fp8_attention(lib, q, k, v, causal, hadamard, signs)
+    assert lib.last_status()[0] == 0
+    scale = 1 / math.sqrt(256)
     if N > 1:
         o_ref, l_ref = A.attention(q, k, v, scale, causal)
         err = errors(o.cpu(), lse.cpu(), o_ref, l_ref)
