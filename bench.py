@@ -326,6 +326,35 @@ def time_shape(B, H, N, d, causal, dev, steps, warmup, world):
             "inputs": "torch.randn bf16 (timing only)"}
 
 
+def time_fp8_shape(B, H, N, d, causal, dev, steps, warmup, world):
+    """TFLOP/s of attn_fwd_fp8 on one shape, the e4m3 operands resident:
+    timing-only inputs (torch.randn bf16 with 0.1 % of the entries scaled by
+    10), Q and K rotated, 128 x d block scales."""
+    from io_aware_attention_02_b200 import binding
+    g = torch.Generator(device=dev).manual_seed(0)
+    xs = []
+    for _ in range(3):
+        x = torch.randn(B, H, N, d, device=dev, dtype=torch.float32, generator=g)
+        hit = torch.rand(B, H, N, d, device=dev, generator=g) < 1e-3
+        xs.append(torch.where(hit, x * 10.0, x).to(torch.bfloat16))
+        del x, hit
+    signs = torch.from_numpy(inputs.hadamard_signs(d, seed=0)).to(dev)
+    q8, qs = binding.quant_fp8(xs[0], hadamard=True, signs=signs)
+    k8, ks = binding.quant_fp8(xs[1], hadamard=True, signs=signs)
+    v8, vs = binding.quant_fp8(xs[2])
+    o = torch.empty_like(xs[0])
+    del xs
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    f = flops(B, H, N, d, causal)
+    n = max(3, min(steps, int(2e13 / f)))
+    ms = timed(lambda: binding.fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, out=o, lse=lse), n, warmup,
+               world) / n
+    return {"tflops": f / (ms * 1e-3) / 1e12, "ms": ms, "steps": n,
+            "pct_of_spec_fp8_peak": 100 * f / (ms * 1e-3) / 1e12 / SPEC_FP8_TFLOPS,
+            "shape": f"B={B},H={H},N={N},d={d},{'causal' if causal else 'non-causal'}",
+            "inputs": "torch.randn bf16 with 0.1% entries x10, quantised once (timing only)"}
+
+
 def run_ours(args, world, rank, local):
     from io_aware_attention_02_b200 import binding
     binding.load()
@@ -407,10 +436,12 @@ def run_ours(args, world, rank, local):
                   flush=True)
         return
 
-    if args.only in ("d64", "d256", "causal", "long"):
+    if args.only in ("d64", "d256", "causal", "long", "fp8d64", "fp8d256"):
         SB, SH, SN, Sd, sc = {"d64": (8, 16, 8192, 64, False), "d256": (2, 16, 8192, 256, False),
-                              "causal": (B, H, N, d, True), "long": (1, 32, 65536, 128, True)}[args.only]
-        r = time_shape(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
+                              "causal": (B, H, N, d, True), "long": (1, 32, 65536, 128, True),
+                              "fp8d64": (8, 16, 8192, 64, False), "fp8d256": (2, 16, 8192, 256, False)}[args.only]
+        timer = time_fp8_shape if args.only.startswith("fp8") else time_shape
+        r = timer(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
         code, where = binding.last_status()
         if code != 0:
             raise RuntimeError(f"kernel status {code} at {where}")
@@ -494,6 +525,10 @@ def run_ours(args, world, rank, local):
             "bf16_d256_B2H16N8192_causal": (2, 16, 8192, 256, True),
             "bf16_long_B1H32N65536_d128_causal": (1, 32, 65536, 128, True)}.items():
         shape_var[name] = time_shape(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
+    for name, (SB, SH, SN, Sd, sc) in {
+            "fp8_e4m3_d64_B2H16N8192": (2, 16, 8192, 64, False),
+            "fp8_e4m3_d256_B2H16N8192": (2, 16, 8192, 256, False)}.items():
+        shape_var[name] = time_fp8_shape(SB, SH, SN, Sd, sc, dev, args.steps, args.warmup, world)
     code, where = binding.last_status()
     if code != 0:
         raise RuntimeError(f"kernel status {code} at {where}")
@@ -674,12 +709,13 @@ def main():
                     help="seconds of CPU work for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["all", "main", "bwd", "decode", "fp8", "quant", "d64", "d256", "causal",
-                                       "long"], default="all",
+                                       "long", "fp8d64", "fp8d256"], default="all",
                     help="main: time only the bf16 non-causal step; bwd: only the fused bf16 "
                          "non-causal backward of the same workload; decode: only the split-KV decode "
                          "variant; fp8 / quant: only the FP8 forward / the FP8 quantisation of Q, K, V; "
                          "d64 (B=8, N=8K), d256 (B=2, N=8K), causal, long (B=1, H=32, N=64K causal): "
-                         "only that bf16 forward (for profiler runs)")
+                         "only that bf16 forward; fp8d64 (B=8, N=8K), fp8d256 (B=2, N=8K): only that FP8 "
+                         "forward (for profiler runs)")
     ap.add_argument("--decode-nk", type=int, default=32768,
                     help="KV length of the --only decode run (smaller for profiler captures)")
     ap.add_argument("--sweep", action="store_true",
