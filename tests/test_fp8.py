@@ -164,6 +164,24 @@ def test_fp8_head_dim_256(lib, causal, hadamard, N):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_fp8_head_dim_256_many_units(lib, causal):
+    """Head dim 256 with several work units per CTA (4 x 16 heads x 8 row
+    tiles = 512 units), sampled rows of three heads against the fp64
+    oracle."""
+    B, H, N = 4, 16, 1024
+    q, k, v = _x(B, H, N, 256, seed=60)
+    signs = inputs.hadamard_signs(256, seed=6)
+    o, lse, _ = _fp8_attention(lib, q, k, v, causal, True, signs)
+    assert lib.last_status()[0] == 0
+    rows = inputs.sample_rows(N, 48, seed=9)
+    scale = 1 / math.sqrt(256)
+    for b, h in [(0, 0), (1, 7), (3, 15)]:
+        o_ref, l_ref = A.attention_head(q[b, h], k[b, h], v[b, h], scale, causal, rows)
+        err = errors(o[b, h][rows].cpu(), lse[b, h][rows].cpu(), o_ref, l_ref)
+        assert err["rmse"] <= FP8_RMSE, (b, h, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_fp8_headline_shape_sampled(lib, causal):
     """B=4, H=16, N=8192, d=128 with outliers; Hadamard on; sampled rows."""
     q, k, v = _x(4, 16, 8192, 128, seed=0)
