@@ -55,7 +55,9 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,  /* head dim or dtype the library does not handle */
   ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned             */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed          */
-  ATTN_ERR_TIMEOUT = 5       /* a kernel wait ran out (read after sync)       */
+  ATTN_ERR_TIMEOUT = 5,      /* a kernel wait ran out (read after sync)       */
+  ATTN_ERR_BOUNDS = 6        /* debug build only: a TMEM or shared-memory
+                                range check failed (read after sync)          */
 } attn_status_t;
 
 typedef enum {
@@ -147,7 +149,8 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
 
 /*
  * attn_last_status -- synchronises `stream`, then reads and clears the
- * current device's status word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT (a kernel
+ * current device's status word.  Returns ATTN_OK, ATTN_ERR_BOUNDS (debug build:
+ * a range check failed), ATTN_ERR_TIMEOUT (a kernel
  * wait ran out; the affected outputs are undefined) or ATTN_ERR_CUDA.
  * `where` (may be NULL) receives 2 ints: the barrier id and block index
  * recorded with the error.
@@ -337,6 +340,11 @@ const char* attn_status_string(attn_status_t s);
  * returns ATTN_OK and attn_last_status() then reports ATTN_ERR_TIMEOUT.  The
  * hook resets itself after one launch.  `wait_limit_ms` (> 0) overrides the
  * wait limit for that launch.  No device fault, trap or hang is involved.
+ * Mode 2 exists in the debug build only (ATTN_ERR_UNSUPPORTED otherwise): the
+ * next attn_fwd launch checks CTA 0's first S load of TMEM as if its columns
+ * were out of range, so attn_last_status() reports ATTN_ERR_BOUNDS (where =
+ * the check's id, 29); the load itself is never out of range: the failed check
+ * skips it, and that launch's outputs are undefined.
  */
 attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms);
 

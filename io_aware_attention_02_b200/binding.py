@@ -16,8 +16,9 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libattn_sm100.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libattn_sm100_debug.so")
 
-ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(6)
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_BOUNDS = range(7)
 ATTN_BF16, ATTN_FP16 = 0, 1
 
 # name -> (restype, argtypes); mirrors include/attn.h
@@ -72,6 +73,23 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def lib() -> ctypes.CDLL:
     return load()
+
+
+def load_debug(path: str = DEBUG_LIB_PATH) -> ctypes.CDLL:
+    """The debug build (``build --debug``: range checks on every TMEM and
+    shared-memory access of the forward kernel, ATTN_ERR_BOUNDS on a failed
+    one), loaded beside the release library with the same signatures.  Call
+    its entry points directly; the wrappers of this module use the release
+    library."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m io_aware_attention_02_b200.build --debug`")
+    dlib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(dlib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return dlib
 
 
 def status_string(code: int) -> str:

@@ -452,12 +452,14 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "kernel wait timed out";
+    case ATTN_ERR_BOUNDS: return "debug bounds check failed";
   }
   return "unknown status";
 }
 
 attn_status_t attn_debug_set_fault(int mode, int wait_limit_ms) {
-  if (mode < 0 || mode > 1 || wait_limit_ms < 0) return ATTN_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 2 || wait_limit_ms < 0) return ATTN_ERR_INVALID_ARG;
+  if (mode == 2 && !ATTN_DEBUG_BOUNDS) return ATTN_ERR_UNSUPPORTED;   // the range checks exist in the debug build only
   std::lock_guard<std::mutex> lock(g_mu);
   g_fault_mode = mode;
   g_fault_limit_ms = wait_limit_ms;
@@ -484,7 +486,8 @@ attn_status_t attn_last_status(void* stream, int* where) {
     where[1] = h[2];
   }
   if (h[0] == 0) return ATTN_OK;
-  return h[0] == ATTN_ERR_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+  if (h[0] == ATTN_ERR_TIMEOUT || h[0] == ATTN_ERR_BOUNDS) return static_cast<attn_status_t>(h[0]);
+  return ATTN_ERR_CUDA;
 }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -705,7 +708,8 @@ extern "C" attn_status_t attn_noalloc_last_status(void* stream, int* where) {
     where[1] = h[2];
   }
   if (h[0] == 0) return ATTN_OK;
-  return h[0] == ATTN_ERR_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+  if (h[0] == ATTN_ERR_TIMEOUT || h[0] == ATTN_ERR_BOUNDS) return static_cast<attn_status_t>(h[0]);
+  return ATTN_ERR_CUDA;
 }
 
 extern "C" int attn_debug_status_allocated(void) {

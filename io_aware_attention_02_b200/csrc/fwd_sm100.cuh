@@ -160,6 +160,14 @@ enum : int {
   kWherePFull = 5, kWhereSFull = 6, kWhereOFull = 7, kWhereDrain = 8
 };
 
+// Range-check ids reported by the debug build (status[1] with kErrBounds):
+// which access of the forward kernel fell outside its region.
+enum : int {
+  kChkQLoad = 21, kChkKvLoad = 22, kChkSOut = 23, kChkSQ = 24, kChkSK = 25, kChkOOut = 26, kChkPIn = 27,
+  kChkVIn = 28, kChkSLoad = 29, kChkPStore = 30, kChkORescale = 31, kChkOLoad = 32, kChkVtSrc = 33,
+  kChkVtDst = 34
+};
+
 // ---------------------------------------------------------------------------
 // Softmax arithmetic helpers
 // ---------------------------------------------------------------------------
@@ -422,9 +430,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, 2 * Cfg::kTileBytes);
         for (int t = 0; t < 2; ++t)
-          for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes, &p.tm_q, q_full,
-                        c * Cfg::kChunkCols, qp * 256 + t * 128, bh % p.H, bh / p.H);
+          for (int c = 0; c < Cfg::kChunks; ++c) {
+            uint8_t* dst = sQ + t * Cfg::kTileBytes + c * Cfg::kChunkBytes;
+            if (smem_range_ok(dst, Cfg::kChunkBytes, smem, Cfg::kOffQ, Cfg::kOffKV, p.status, kChkQLoad))
+              tma_load_4d(dst, &p.tm_q, q_full, c * Cfg::kChunkCols, qp * 256 + t * 128, bh % p.H, bh / p.H);
+          }
         for (int j = 0; j < n1 && ok; ++j) {
           for (int which = 0; which < 2; ++which, ++kv_iter) {
             const uint32_t s = kv_iter % S;
@@ -436,9 +446,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
             }
             mbar_arrive_expect_tx(kv_full + s, Cfg::kTileBytes);
             const CUtensorMap* map = which == 0 ? &p.tm_k : &p.tm_v;
-            for (int c = 0; c < Cfg::kChunks; ++c)
-              tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
-                          c * Cfg::kChunkCols, j * 128, bh % p.H, bh / p.H);
+            for (int c = 0; c < Cfg::kChunks; ++c) {
+              uint8_t* dst = sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes;
+              if (smem_range_ok(dst, Cfg::kChunkBytes, smem, Cfg::kOffKV, Cfg::kOffVt, p.status, kChkKvLoad))
+                tma_load_4d(dst, map, kv_full + s, c * Cfg::kChunkCols, j * 128, bh % p.H, bh / p.H);
+            }
           }
         }
       }
@@ -477,6 +489,13 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       auto issue_s = [&](int t, uint32_t kstage) {
         const uint64_t a0 = dQ + static_cast<uint64_t>((t * Cfg::kTileBytes) >> 4);
         const uint64_t b0 = dK + static_cast<uint64_t>((kstage * Cfg::kTileBytes) >> 4);
+        if (!tmem_range_ok(tmem + Cfg::kColS + t * 128, tmem, 128, Cfg::kColS + t * 128, Cfg::kColS + t * 128 + 128,
+                           p.status, kChkSOut) ||
+            !smem_range_ok(sQ + t * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffQ, Cfg::kOffKV, p.status,
+                           kChkSQ) ||
+            !smem_range_ok(sKV + kstage * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffVt,
+                           p.status, kChkSK))
+          return;
 #pragma unroll
         for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
           // K-major, kSwz-byte swizzle: each product consumes 32 bytes of the
@@ -491,12 +510,22 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
       auto issue_pv_half = [&](int t, uint32_t vstage, int h, bool acc) {
         const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);  // stage or Vt buffer
         constexpr int kSteps = 64 / Cfg::kKeysPerMma;
+        if (!tmem_range_ok(tmem + Cfg::kColO + t * D, tmem, D, Cfg::kColO + t * D, Cfg::kColO + (t + 1) * D, p.status,
+                           kChkOOut) ||
+            !(VT ? smem_range_ok(sVt + vstage * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffVt,
+                                 Cfg::kOffVt + Cfg::kVtBytes, p.status, kChkVIn)
+                 : smem_range_ok(sKV + vstage * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffVt,
+                                 p.status, kChkVIn)))
+          return;
 #pragma unroll
         for (int kk = h * kSteps; kk < (h + 1) * kSteps; ++kk) {
           // P_t: 128 rows x 128 keys packed in TMEM (32 bytes = 8 columns per
           // product).  V_j: MN-major (head dim contiguous), kKeysPerMma keys
           // = kKeysPerMma swizzled rows of kSwz bytes per product.
           const uint32_t voff = VT ? ((kk * 32) >> 4) : ((kk * Cfg::kKeysPerMma * kSwz) >> 4);
+          if (!tmem_range_ok(tmem + Cfg::kColS + t * 128 + kk * 8, tmem, 8, Cfg::kColS + t * 128,
+                             Cfg::kColS + t * 128 + 64, p.status, kChkPIn))
+            continue;
           mma_ts(tmem + Cfg::kColO + t * D, tmem + Cfg::kColS + t * 128 + kk * 8,
                  b0 + voff, idesc_o, (acc || kk > 0) ? 1u : 0u, kF8);
         }
@@ -639,7 +668,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         if (!__all_sync(0xffffffffu, w)) *abort_flag = 1;
         named_bar_sync(3, 64);
         if (*abort_flag) { ok = false; break; }
-        transpose_v_tile_e4m3(sKV + (iv % S) * Cfg::kTileBytes, sVt + b * Cfg::kTileBytes, tt);
+        if (smem_range_ok(sKV + (iv % S) * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffVt, p.status,
+                          kChkVtSrc) &&
+            smem_range_ok(sVt + b * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffVt, Cfg::kOffVt + Cfg::kVtBytes,
+                          p.status, kChkVtDst))
+          transpose_v_tile_e4m3(sKV + (iv % S) * Cfg::kTileBytes, sVt + b * Cfg::kTileBytes, tt);
         // generic-proxy shared-memory writes, read next by the tensor core
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         named_bar_sync(3, 64);
@@ -707,7 +740,17 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
-          tmem_ld32(tS + cc * 32, r);
+#if ATTN_DEBUG_BOUNDS
+          // test hook (fault mode 2): CTA 0's first S load is checked as if it
+          // were 512 columns further on, so that check fails; the load itself
+          // is not shifted, and the failed check skips it
+          const uint32_t shift = (p.fault == 2 && blockIdx.x == 0 && k == 0 && j == 0 && cc == 0) ? 512u : 0u;
+#else
+          constexpr uint32_t shift = 0u;
+#endif
+          if (tmem_range_ok(tS + cc * 32 + shift, tmem, 32, Cfg::kColS + t * 128, Cfg::kColS + t * 128 + 128,
+                            p.status, kChkSLoad))
+            tmem_ld32(tS + cc * 32, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
         }
@@ -741,6 +784,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
 #pragma unroll 1
           for (int cc = 0; cc < D / 16; ++cc) {
             uint32_t r[16];
+            if (!tmem_range_ok(tO + cc * 16, tmem, 16, Cfg::kColO + t * D, Cfg::kColO + (t + 1) * D, p.status,
+                               kChkORescale))
+              continue;
             tmem_ld16(tO + cc * 16, r);
             tmem_wait_ld();
             tmem_reg_fence(r);
@@ -758,8 +804,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
         float sum = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          sum += need_mask ? exp_pack_half<kF8, T, false>(s, h, c, -m, pgain, tS)
-                           : exp_pack_half<kF8, T, true>(s, h, c, -m, pgain, tS);
+          if (tmem_range_ok(tS + (kF8 ? 16 : 32) * h, tmem, kF8 ? 16 : 32, Cfg::kColS + t * 128,
+                            Cfg::kColS + t * 128 + 64, p.status, kChkPStore))
+            sum += need_mask ? exp_pack_half<kF8, T, false>(s, h, c, -m, pgain, tS)
+                             : exp_pack_half<kF8, T, true>(s, h, c, -m, pgain, tS);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(p_full + 2 * t + h);
@@ -782,7 +830,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_sm100_kernel(const __grid_con
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];
-        tmem_ld32(tO + cc * 32, r);
+        if (tmem_range_ok(tO + cc * 32, tmem, 32, Cfg::kColO + t * D, Cfg::kColO + (t + 1) * D, p.status, kChkOLoad))
+          tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
         tmem_reg_fence(r);
         uint32_t pk[16];

@@ -14,13 +14,52 @@ namespace attn {
 // [0] error code (0 = ok), [1] where (role / barrier id), [2] blockIdx.x,
 // [3] reserved.
 // ----------------------------------------------------------------------------
-enum : int { kErrTimeout = 5 };
+enum : int { kErrTimeout = 5, kErrBounds = 6 };
 
 __device__ __forceinline__ void report_error(int* status, int code, int where) {
   if (status != nullptr && atomicCAS(status, 0, code) == 0) {
     status[1] = where;
     status[2] = blockIdx.x;
   }
+}
+
+// ----------------------------------------------------------------------------
+// Range checks of the debug build (compiled with ATTN_DEBUG_BOUNDS=1).  Before
+// a TMEM access the column range [col, col + ncols) relative to the
+// allocation's base must lie in [lo, hi) and the lane offset must be one of
+// the four 32-lane quarters; before a shared-memory access the byte range must
+// lie in [lo, hi) bytes from `base` and start on a 16-byte boundary.  A failed
+// check records kErrBounds with the check's id in the status word and returns
+// false, and the caller skips the access.  In the release build both return
+// true and compile to nothing.
+// ----------------------------------------------------------------------------
+#ifndef ATTN_DEBUG_BOUNDS
+#define ATTN_DEBUG_BOUNDS 0
+#endif
+
+__device__ __forceinline__ bool tmem_range_ok(uint32_t taddr, uint32_t tmem_base, int ncols, int lo, int hi,
+                                              int* status, int where) {
+#if ATTN_DEBUG_BOUNDS
+  const int col = static_cast<int>(taddr & 0xffffu) - static_cast<int>(tmem_base & 0xffffu);
+  const int lane = static_cast<int>(taddr >> 16) - static_cast<int>(tmem_base >> 16);
+  if (col < lo || col + ncols > hi || lane < 0 || lane > 96 || (lane & 31) != 0) {
+    report_error(status, kErrBounds, where);
+    return false;
+  }
+#endif
+  return true;
+}
+
+__device__ __forceinline__ bool smem_range_ok(const void* ptr, int bytes, const void* base, int lo, int hi,
+                                              int* status, int where) {
+#if ATTN_DEBUG_BOUNDS
+  const long long off = static_cast<const uint8_t*>(ptr) - static_cast<const uint8_t*>(base);
+  if (off < lo || off + bytes > hi || (off & 15) != 0) {
+    report_error(status, kErrBounds, where);
+    return false;
+  }
+#endif
+  return true;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

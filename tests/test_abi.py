@@ -220,6 +220,8 @@ def test_debug_hook_validation(lib):
     assert lib.attn_debug_set_ablation(2) == binding.ATTN_ERR_INVALID_ARG
     assert lib.attn_debug_set_ablation(-1) == binding.ATTN_ERR_INVALID_ARG
     assert lib.attn_debug_set_fault(0, 0) == binding.ATTN_OK
+    # mode 2 (a planted range-check failure) exists in the debug build only
+    assert lib.attn_debug_set_fault(2, 0) == binding.ATTN_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_cpu_tensors():
@@ -227,3 +229,18 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.fwd(x, x, x)
+
+
+def test_debug_build_exports_the_same_boundary():
+    """The debug build (range checks in the forward kernel) is the same C ABI:
+    it loads beside the release library, exports every declared entry point,
+    and names the status code its checks report."""
+    from io_aware_attention_02_b200 import build
+    build.build(debug=True)
+    dlib = binding.load_debug()
+    for name in _declared():
+        assert hasattr(dlib, name), name
+    assert dlib.attn_status_string(binding.ATTN_ERR_BOUNDS) == b"debug bounds check failed"
+    assert binding.load().attn_status_string(binding.ATTN_ERR_BOUNDS) == b"debug bounds check failed"
+    assert dlib.attn_debug_set_fault(2, 0) == binding.ATTN_OK     # accepted here; reset it
+    assert dlib.attn_debug_set_fault(0, 0) == binding.ATTN_OK
