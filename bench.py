@@ -50,7 +50,7 @@ METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense BF16/FP8 tensor peak"
 # above, from the ncu DRAM capture of this kernel (`ncu --metrics
 # dram__bytes_read.sum,dram__bytes_write.sum`), keyed by the sha256 of the
 # kernel source it was measured on: reported only while the source is unchanged.
-TRAFFIC = {"82772d472c985198": 517491968}
+TRAFFIC = {"94b24a8bc775b81d": 518538496}
 
 
 def flops(B, H, N, d, causal):
