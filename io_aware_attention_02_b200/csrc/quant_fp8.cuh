@@ -9,19 +9,18 @@
 // item 3.  The rotation leaves Q K^T unchanged because it is orthogonal.
 //
 // Streaming kernel: 2 bytes read and 1 byte written per element, meant to run
-// at HBM bandwidth.  Persistent CTAs of 128 * D/64 threads (three per SM at
-// D = 64, two at 128, one at 256) walk the blocks of 128 rows of one (batch,
-// head) in a strided order.
+// at HBM bandwidth.  Persistent CTAs of 256 threads (three per SM) at D = 64,
+// 256 (two per SM) at 128 and 512 (one per SM) at 256 walk the blocks of 128
+// rows of one (batch, head) in a strided order.
 // Thread 0 keeps a ring of kStages blocks in flight: each block arrives by
 // TMA (tile loads of 64 columns x 128 rows, 128-byte swizzle, rows past N
-// zero-filled).  A thread owns 64 columns of one row (the D/64 threads of a
-// row are neighbouring lanes): it reads them from shared memory (the
-// swizzle spreads a warp's 16-byte reads over all banks), applies the signs
-// (a flip of the bf16 sign bits), runs the six butterfly stages of the fast
-// Walsh-Hadamard transform that stay inside its 64 values in registers and,
-// at d = 128 and 256, the remaining stages with its neighbours by one lane
-// shuffle per value and stage; then it scales by 1/sqrt(D) and takes its
-// amax.  The block's amax
+// zero-filled).  A thread owns kVals columns of one row (32 at D = 64, 64
+// otherwise; the threads of a row are neighbouring lanes): it reads them from
+// shared memory (the swizzle spreads a warp's 16-byte reads over all banks),
+// applies the signs (a flip of the bf16 sign bits), runs the butterfly stages
+// of the fast Walsh-Hadamard transform that stay inside its values in
+// registers and the remaining stages with its neighbours by one lane shuffle
+// per value and stage; then it scales by 1/sqrt(D) and takes its amax.  The block's amax
 // needs every row, so the CTA meets at one barrier per block; that barrier
 // also tells thread 0 that the block's buffer has been read and may be
 // refilled.  Each thread then rounds its 64 values to e4m3 into one of two
@@ -57,20 +56,25 @@ struct QuantCfg {
   // 2 x 64 + 2 x 32 KiB and one CTA at D = 256
   static constexpr int kStages = D == 64 ? 3 : 2;
   static constexpr int kMinBlocks = D == 64 ? 3 : (D == 128 ? 2 : 1);
+  // values of a row per thread: 32 at D = 64 (twice the warps of 64 values,
+  // measured 10 % faster there), 64 otherwise (32 measured 6 % slower at
+  // D = 128: one more lane-shuffle stage per value)
+  static constexpr int kVals = D == 64 ? 32 : 64;
   static constexpr int kOutBytes = kRows * D;                // one block of codes
   // the codes of a block go out in column chunks of at most 128 bytes (the
   // widest swizzled box): one chunk up to D = 128, two at D = 256
   static constexpr int kOutChunkCols = D < 128 ? D : 128;
   static constexpr int kOutChunks = D / kOutChunkCols;
-  static constexpr int kTpr = D / 64;                        // threads per row
+  static constexpr int kTpr = D / kVals;                     // threads per row
+  static constexpr int kPieces = kVals / 8;                  // 16-byte input pieces per thread
   static constexpr int kThreads = 128 * kTpr;
   static constexpr int kWarps = kThreads / 32;
   static constexpr int kOutOff = kStages * kTileBytes;     // [2] staging tiles
   static constexpr int kBarOff = kOutOff + 2 * kOutBytes;
   static constexpr int kAbortOff = kBarOff + 64;
-  static constexpr int kRedOff = kBarOff + 128;             // float [2][kWarps <= 8]
-  static constexpr int kSgnOff = kBarOff + 256;             // uint32 [D / 2]: sign bits per bf16 pair
-  static_assert(2 * kWarps * 4 <= 128, "amax slots overflow their region");
+  static constexpr int kRedOff = kBarOff + 128;             // float [2][kWarps <= 32]
+  static constexpr int kSgnOff = kBarOff + 384;             // uint32 [D / 2]: sign bits per bf16 pair
+  static_assert(2 * kWarps * 4 <= 256, "amax slots overflow their region");
   static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
   static constexpr int kSmem = kSgnOff + 2 * D + 1024;      // + alignment slack for the swizzle
   static_assert(kStages * 8 <= 64, "barriers overflow their slot");
@@ -114,7 +118,7 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
 
   const int tid = threadIdx.x;
   const int r = tid / C::kTpr;            // row within the block
-  const int hc = tid % C::kTpr;           // 64-column chunk of that row
+  const int hc = tid % C::kTpr;           // which kVals columns of that row
   const int warp = tid >> 5;
 
   // Block t = bh * n_blocks + blk: rows [128 blk, 128 blk + 128) of head bh.
@@ -163,17 +167,18 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
                               kWhereQuantFull, p.wait_limit_ns);
     const int row0 = (t % p.n_blocks) * C::kRows;
 
-    // this thread's 64 values from the swizzled tile (16-byte piece q of the
+    // this thread's kVals values, columns kVals*hc .. (16-byte piece q of a
     // 64-column chunk sits at piece q ^ (row % 8) of the row's 128 bytes),
-    // held as 32 pairs y[i] = (value 2i, value 2i + 1)
-    float2 y[32];
-    const uint8_t* tile = smem + stage * C::kTileBytes + hc * C::kChunkBytes + r * 128;
+    // held as pairs y[i] = (value 2i, value 2i + 1)
+    float2 y[C::kVals / 2];
+    const uint8_t* tile = smem + stage * C::kTileBytes + (hc * C::kVals / 64) * C::kChunkBytes + r * 128;
+    const int qbase = (hc * C::kVals % 64) / 8;   // first piece of this thread in its chunk row
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < C::kPieces; ++q) {
       uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (ok) raw = *reinterpret_cast<const uint4*>(tile + ((q ^ (r & 7)) << 4));
-      if (rot) {   // four words shared by all threads of a chunk: a broadcast read
-        const uint4 m = reinterpret_cast<const uint4*>(sgn)[hc * 8 + q];
+      if (ok) raw = *reinterpret_cast<const uint4*>(tile + (((qbase + q) ^ (r & 7)) << 4));
+      if (rot) {   // four words shared by the threads of this column range: a broadcast read
+        const uint4 m = reinterpret_cast<const uint4*>(sgn)[hc * C::kPieces + q];
         raw.x ^= m.x; raw.y ^= m.y; raw.z ^= m.z; raw.w ^= m.w;
       }
       y[q * 4 + 0] = unpack2<__nv_bfloat16>(raw.x);
@@ -185,18 +190,18 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
       // fast Walsh-Hadamard transform, one rounding per output of each stage
       // (index bit 0 first): bit 0 pairs the two values of a pair ...
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < C::kVals / 2; ++i) {
         const float a = y[i].x, b = y[i].y;
         y[i] = make_float2(a + b, a - b);
       }
-      // ... bits 1 to 5 pair whole pairs: one paired add and one paired
-      // multiply-add by -1 (an exact negation, then the one rounding of
-      // a - b) per two butterflies ...
+      // ... the next bits up to log2(kVals) - 1 pair whole pairs: one paired
+      // add and one paired multiply-add by -1 (an exact negation, then the
+      // one rounding of a - b) per two butterflies ...
       const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
-      for (int h = 1; h < 32; h <<= 1) {
+      for (int h = 1; h < C::kVals / 2; h <<= 1) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < C::kVals / 2; ++i) {
           if ((i & h) == 0) {
             const float2 a = y[i], b = y[i | h];
             y[i] = __fadd2_rn(a, b);
@@ -204,15 +209,15 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
           }
         }
       }
-      // ... and the index bits above 5 (bit 6 + s is bit s of the chunk
-      // index hc) with the lane that differs in that bit (lower chunk:
-      // y + other; upper chunk: other - y)
+      // ... and the index bits above (bit log2(kVals) + s is bit s of hc)
+      // with the lane that differs in that bit (lower half: y + other;
+      // upper half: other - y)
 #pragma unroll
       for (int sb = 1; sb < C::kTpr; sb <<= 1) {
         const float sg = (hc & sb) == 0 ? 1.f : -1.f;
         const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < C::kVals / 2; ++i) {
           const float2 other = make_float2(__shfl_xor_sync(0xffffffffu, y[i].x, sb),
                                            __shfl_xor_sync(0xffffffffu, y[i].y, sb));
           y[i] = __ffma2_rn(sg2, y[i], other);
@@ -220,11 +225,11 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
       }
       const float2 norm2 = make_float2(norm, norm);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = __fmul2_rn(y[i], norm2);
+      for (int i = 0; i < C::kVals / 2; ++i) y[i] = __fmul2_rn(y[i], norm2);
     }
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmax3(amax, fabsf(y[i].x), fabsf(y[i].y));
+    for (int i = 0; i < C::kVals / 2; ++i) amax = fmax3(amax, fabsf(y[i].x), fabsf(y[i].y));
 
     // Block amax.  The slots alternate between blocks: a warp writes slot
     // set (it & 1) again only two barriers later, after every warp has read it.
@@ -260,18 +265,19 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads, QuantCfg<D>::kMinBlocks
     const float r_lo = __fmul_rn(rc, 1.f - 0x1p-20f), r_hi = __fmul_rn(rc, 1.f + 0x1p-20f);
     const float2 r_lo2 = make_float2(r_lo, r_lo), r_hi2 = make_float2(r_hi, r_hi);
 
-    // this thread's 64 codes: 16-byte pieces hc*4 + g of the row, in column
-    // chunk (hc*64) / kOutChunkCols, swizzled the way the TMA store reads
-    // them (the swizzle XORs the 16-byte piece index within the chunk row
-    // with address bits 7 and up: row % 8 for 128-byte rows, (row / 2) % 4
-    // for 64-byte rows)
+    // this thread's kVals codes: 16-byte pieces kVals*hc/16 + g of the row,
+    // in column chunk (kVals*hc) / kOutChunkCols, swizzled the way the TMA
+    // store reads them (the swizzle XORs the 16-byte piece index within the
+    // chunk row with address bits 7 and up: row % 8 for 128-byte rows,
+    // (row / 2) % 4 for 64-byte rows)
     const int xr = D >= 128 ? (r & 7) : ((r >> 1) & 3);
     constexpr int kPiecesPerChunkRow = C::kOutChunkCols / 16;
-    const int piece0 = (hc * 4) % kPiecesPerChunkRow;
-    uint8_t* orow = out_tiles + (it & 1) * C::kOutBytes + ((hc * 4) / kPiecesPerChunkRow) * (C::kRows * C::kOutChunkCols) +
+    const int opiece = hc * C::kVals / 16;
+    const int piece0 = opiece % kPiecesPerChunkRow;
+    uint8_t* orow = out_tiles + (it & 1) * C::kOutBytes + (opiece / kPiecesPerChunkRow) * (C::kRows * C::kOutChunkCols) +
                     r * C::kOutChunkCols;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 0; g < C::kVals / 16; ++g) {
       uint4 v;
       v.x = quant4_e4m3(y[8 * g], y[8 * g + 1], s, r_lo2, r_hi2, fast);
       v.y = quant4_e4m3(y[8 * g + 2], y[8 * g + 3], s, r_lo2, r_hi2, fast);
