@@ -127,8 +127,10 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * Cfg::kChunkCols, qt * 128, bh % p.H,
-                      bh / p.H);
+          if (smem_range_ok(sQ + c * Cfg::kChunkBytes, Cfg::kChunkBytes, smem, Cfg::kOffQ, Cfg::kOffKV, p.status,
+                            kChkQLoad))
+            tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * Cfg::kChunkCols, qt * 128, bh % p.H,
+                        bh / p.H);
         for (int q = 0; q < 2 * n && ok; ++q, ++kv_iter) {
           // q -> (K or V, key tile j), inverse of seq_k / seq_v
           const bool is_v = (q == 2 * n - 1) || (q > 0 && (q & 1) == 0);
@@ -143,8 +145,10 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
           mbar_arrive_expect_tx(kv_full + s, Cfg::kTileBytes);
           const CUtensorMap* map = is_v ? &p.tm_v : &p.tm_k;
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
-                        c * Cfg::kChunkCols, j * 128, bh % p.H, bh / p.H);
+            if (smem_range_ok(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, Cfg::kChunkBytes, smem, Cfg::kOffKV,
+                              Cfg::kOffBar, p.status, kChkKvLoad))
+              tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s,
+                          c * Cfg::kChunkCols, j * 128, bh % p.H, bh / p.H);
         }
       }
       if (!ok) {
@@ -170,6 +174,11 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
 
       auto issue_s = [&](int buf, uint32_t kstage) {
         const uint64_t b0 = dK + static_cast<uint64_t>((kstage * Cfg::kTileBytes) >> 4);
+        if (!tmem_range_ok(tmem + buf * 128, tmem, 128, buf * 128, buf * 128 + 128, p.status, kChkSOut) ||
+            !smem_range_ok(sQ, Cfg::kTileBytes, smem, Cfg::kOffQ, Cfg::kOffKV, p.status, kChkSQ) ||
+            !smem_range_ok(sKV + kstage * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffBar,
+                           p.status, kChkSK))
+          return;
 #pragma unroll
         for (int kk = 0; kk < D / Cfg::kKeysPerMma; ++kk) {
           // 32 bytes of the head dim per product, four per 128-byte chunk row
@@ -183,9 +192,15 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
       auto pv = [&](int buf, uint32_t vstage, bool acc) -> bool {
         const uint64_t b0 = dV + static_cast<uint64_t>((vstage * Cfg::kTileBytes) >> 4);
         constexpr int kSteps = 64 / Cfg::kKeysPerMma;
+        const bool in_range =
+            tmem_range_ok(tmem + Cfg::kColO, tmem, D, Cfg::kColO, Cfg::kColO + D, p.status, kChkOOut) &&
+            tmem_range_ok(tmem + buf * 128, tmem, 64, buf * 128, buf * 128 + 64, p.status, kChkPIn) &&
+            smem_range_ok(sKV + vstage * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffBar, p.status,
+                          kChkVIn);
         for (int h = 0; h < 2; ++h) {
           if (!mbar_wait(p_full + h, p_cnt & 1, p.status, abort_flag, kWherePFull, lim)) return false;
           tc_fence_after();
+          if (!in_range) continue;
 #pragma unroll
           for (int kk = kSteps * h; kk < kSteps * (h + 1); ++kk)
             mma_ts(tmem + Cfg::kColO, tmem + buf * 128 + kk * 8, b0 + ((kk * Cfg::kKeysPerMma * 128) >> 4),
@@ -298,7 +313,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
-          tmem_ld32(tS + cc * 32, r);
+          if (tmem_range_ok(tS + cc * 32, tmem, 32, buf * 128, buf * 128 + 128, p.status, kChkSLoad))
+            tmem_ld32(tS + cc * 32, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
         }
@@ -331,6 +347,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t r[32];
+              if (!tmem_range_ok(tO + cc * 32, tmem, 32, Cfg::kColO, Cfg::kColO + D, p.status, kChkORescale))
+                continue;
               tmem_ld32(tO + cc * 32, r);
               tmem_wait_ld();
               tmem_reg_fence(r);
@@ -342,11 +360,13 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
             }
           }
         }
-        store_p_half<kF8>(tS, 0, pk0);
+        const bool p_ok = tmem_range_ok(tS, tmem, 64, buf * 128, buf * 128 + 64, p.status, kChkPStore);
+        if (p_ok) store_p_half<kF8>(tS, 0, pk0);
         tc_fence_before();
         mbar_arrive(p_full + 0);
-        sum += need_mask ? exp_pack_half<kF8, T, false>(s, 1, c, -m, pgain, tS)
-                         : exp_pack_half<kF8, T, true>(s, 1, c, -m, pgain, tS);
+        if (p_ok)
+          sum += need_mask ? exp_pack_half<kF8, T, false>(s, 1, c, -m, pgain, tS)
+                           : exp_pack_half<kF8, T, true>(s, 1, c, -m, pgain, tS);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + 1);
@@ -372,7 +392,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_sm100_d256_kernel(const __gri
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];
-        tmem_ld32(tO + cc * 32, r);
+        if (tmem_range_ok(tO + cc * 32, tmem, 32, Cfg::kColO, Cfg::kColO + D, p.status, kChkOLoad))
+          tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
         tmem_reg_fence(r);
         uint32_t pk[16];

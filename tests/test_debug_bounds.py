@@ -1,8 +1,9 @@
 """GPU runs of the debug build (every TMEM column range and shared-memory
-byte range of the forward kernel checked before use; a failed check reports
+byte range of the forward kernels checked before use; a failed check reports
 ATTN_ERR_BOUNDS and skips the access) on small cases of each variant of the
-kernel: no check fails, and the outputs are bit-identical to the release
-build's on the same inputs."""
+two-tile kernel (head dims 64, 128) and the one-tile kernel (200 padded to
+256, 256), bf16 and e4m3: no check fails, and the outputs are bit-identical
+to the release build's on the same inputs."""
 
 import math
 
@@ -44,7 +45,7 @@ def _fwd(l, q, k, v, causal):
     return o, lse
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 200, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 200, 700])
 def test_bf16_debug_build_matches_release(lib, dlib, d, causal, N):
@@ -55,7 +56,7 @@ def test_bf16_debug_build_matches_release(lib, dlib, d, causal, N):
     assert torch.equal(o, od) and torch.equal(lse, lsed)
 
 
-@pytest.mark.parametrize("d,vt", [(64, 0), (128, 0), (128, 1)])
+@pytest.mark.parametrize("d,vt", [(64, 0), (128, 0), (128, 1), (256, 0)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_fp8_debug_build_matches_release(lib, dlib, d, vt, causal):
     N = 600
