@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
         for (int c = 0; c < Cfg::kChunks; ++c)
-          tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * 64, qt * 128, h, b);
+          if (smem_range_ok(sQ + c * Cfg::kChunkBytes, Cfg::kChunkBytes, smem, 0, Cfg::kOffKV, p.status, kChkQLoad))
+            tma_load_4d(sQ + c * Cfg::kChunkBytes, &p.tm_q, q_full, c * 64, qt * 128, h, b);
         ++unit_iter;
         // consumption order: K0, K1, then V(jj), K(jj + 2) for jj = 0, 1, ...
         auto load = [&](const CUtensorMap* map, int j) -> bool {
@@ -166,7 +167,9 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
             return false;
           mbar_arrive_expect_tx(kv_full + s, Cfg::kTileBytes);
           for (int c = 0; c < Cfg::kChunks; ++c)
-            tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s, c * 64, j * 128, h, b);
+            if (smem_range_ok(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, Cfg::kChunkBytes, smem, Cfg::kOffKV,
+                              Cfg::kOffBar, p.status, kChkKvLoad))
+              tma_load_4d(sKV + s * Cfg::kTileBytes + c * Cfg::kChunkBytes, map, kv_full + s, c * 64, j * 128, h, b);
           ++kv_iter;
           return true;
         };
@@ -206,8 +209,12 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
       // S(buffer b) = Q K^T from ring stage s
       auto issue_s = [&](int b, uint32_t s) {
         const uint64_t b0 = dK + static_cast<uint64_t>((s * Cfg::kTileBytes) >> 4);
+        const bool in_range =
+            tmem_range_ok(tmem + b * 128, tmem, 128, b * 128, b * 128 + 128, p.status, kChkSOut) &&
+            smem_range_ok(sKV + s * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffBar, p.status,
+                          kChkSK);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16 && in_range; ++kk) {
           const uint32_t off = ((kk >> 2) * Cfg::kChunkBytes + (kk & 3) * 32) >> 4;
           mma_ss(tmem + b * 128, dQ + off, b0 + off, idesc_s, kk > 0, false);
         }
@@ -243,8 +250,13 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
           if (!ok) break;
           // O += P V: P packed over S buffer b (8 columns per 16 keys), V MN-major
           const uint64_t b0 = dV + static_cast<uint64_t>((sv * Cfg::kTileBytes) >> 4);
+          const bool pv_in_range =
+              tmem_range_ok(tmem + Cfg::kColO, tmem, D, Cfg::kColO, Cfg::kColO + D, p.status, kChkOOut) &&
+              tmem_range_ok(tmem + b * 128, tmem, 64, b * 128, b * 128 + 64, p.status, kChkPIn) &&
+              smem_range_ok(sKV + sv * Cfg::kTileBytes, Cfg::kTileBytes, smem, Cfg::kOffKV, Cfg::kOffBar, p.status,
+                            kChkVIn);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 8 && pv_in_range; ++kk)
             mma_ts(tmem + Cfg::kColO, tmem + b * 128 + kk * 8, b0 + ((kk * 16 * 128) >> 4), idesc_o,
                    (jj > 0 || kk > 0) ? 1u : 0u, false);
           mma_commit(kv_empty + sv);
@@ -301,7 +313,8 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t rr[32];
-            tmem_ld32(tS + cc * 32, rr);
+            if (tmem_range_ok(tS + cc * 32, tmem, 32, b * 128, b * 128 + 128, p.status, kChkSLoad))
+              tmem_ld32(tS + cc * 32, rr);
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(rr[i]);
           }
@@ -330,6 +343,8 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t rr[32];
+              if (!tmem_range_ok(tO + cc * 32, tmem, 32, Cfg::kColO, Cfg::kColO + D, p.status, kChkORescale))
+                continue;
               tmem_ld32(tO + cc * 32, rr);
               tmem_wait_ld();
               tmem_reg_fence(rr);
@@ -345,8 +360,9 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
           float sum = 0.f;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            sum += need_mask ? exp_pack_half<false, T, false>(s, h, c, neg_m, 1.0f, tS)
-                             : exp_pack_half<false, T, true>(s, h, c, neg_m, 1.0f, tS);
+            if (tmem_range_ok(tS + 32 * h, tmem, 32, b * 128, b * 128 + 64, p.status, kChkPStore))
+              sum += need_mask ? exp_pack_half<false, T, false>(s, h, c, neg_m, 1.0f, tS)
+                               : exp_pack_half<false, T, true>(s, h, c, neg_m, 1.0f, tS);
           l = l * alpha + sum;
           tmem_wait_st();
         }
@@ -368,7 +384,8 @@ __global__ void __launch_bounds__(256, 1) attn_splitkv_kernel(const __grid_const
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t rr[32];
-        tmem_ld32(tO + cc * 32, rr);
+        if (tmem_range_ok(tO + cc * 32, tmem, 32, Cfg::kColO, Cfg::kColO + D, p.status, kChkOLoad))
+          tmem_ld32(tO + cc * 32, rr);
         tmem_wait_ld();
         tmem_reg_fence(rr);
         if (row < p.Nq) {

@@ -92,3 +92,31 @@ def test_planted_range_failure_is_reported(lib, dlib):
     od, lsed = _fwd(dlib, q, k, v, False)
     assert _status(dlib) == (0, [0, 0])
     assert torch.equal(o, od) and torch.equal(lse, lsed)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1000), (200, 700)])
+def test_splitkv_debug_build_matches_release(lib, dlib, d, causal, Nq, Nk):
+    """The split-KV kernel's range checks (its Q tile, K/V ring, S buffers,
+    O and P columns) on decode and prefill-against-cache shapes."""
+    B, H = 2, 3
+    g = torch.Generator().manual_seed(Nq + d)
+    q = torch.randn(B, H, Nq, d, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16).cuda()
+    ns = 3
+    ws_bytes = int(binding.load().attn_fwd_splitkv_workspace_bytes(B, H, Nq, d, ns))
+    outs = []
+    for l in (binding.load(), dlib):
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        code = l.attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Nq,
+                                  Nk, d, 1 / math.sqrt(d), int(causal), ns, binding.ATTN_BF16, ws.data_ptr(),
+                                  ws_bytes, torch.cuda.current_stream().cuda_stream)
+        assert code == 0, code
+        torch.cuda.synchronize()
+        outs.append((o, lse))
+    assert _status(dlib) == (0, [0, 0])
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
